@@ -1,0 +1,389 @@
+#!/usr/bin/env python
+"""Benchmark of the B200 SVG-EAR sparse-attention operator (one attention layer).
+
+A step is one svgear_forward over the whole layer: k-means of queries and keys,
+permutation, block error, routing and hybrid attention, on synthetic
+video-DiT-shaped inputs already resident in HBM.  The headline value is the
+dense-equivalent throughput 4*H*N^2*d / layer time; the line also carries the
+per-layer ms, the executed-pair throughput of the attention stage, the routing
+overhead and the per-stage breakdown.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--config wan]
+  python bench.py --impl reference ...   # the CPU oracle on a bounded sample
+
+With N > 1 (torchrun), every rank runs its own full layer (heads are
+independent problems; no collective on the data path) and the value is the
+work of all ranks over the slowest rank's time ("scaling": "weak").
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "SVG-EAR attn layer ms & dense-equiv TFLOP/s at 75.6K tok; routing overhead %"
+UNIT = "TFLOP/s (dense-equivalent 4*H*N^2*d per layer)"
+
+
+def _args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=5)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--config", default="wan")
+    ap.add_argument("--rho", type=float, default=None)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    return ap.parse_args()
+
+
+def _workload(cfg, rho):
+    grid = "x".join(map(str, cfg.grid)) if cfg.grid else "uniform"
+    return (f"{cfg.name}: H={cfg.H}, N={cfg.N} ({grid}), d={cfg.d}, {cfg.dtype}, Cq={cfg.Cq}, "
+            f"Ck={cfg.Ck}, rho={rho}, kmeans iters={cfg.iters}, G={cfg.G} latent centers, "
+            f"sigma={cfg.sigma}")
+
+
+def _gen_head(args):
+    name, h = args
+    from clustered_sparse_attention_flash_b200 import synth
+    cfg = synth.CONFIGS[name]
+    q, k, v, _ = synth.make_head(cfg, h)
+    iq = synth.forgy_init(cfg, q, h, 0, cfg.Cq)
+    ik = synth.forgy_init(cfg, k, h, 1, cfg.Ck)
+    return q, k, v, iq, ik
+
+
+def generate(cfg):
+    """All heads of the config, generated in a spawn pool (before any CUDA)."""
+    import multiprocessing as mp
+    import numpy as np
+    from clustered_sparse_attention_flash_b200 import synth
+    synth.logit_alpha(cfg)
+    n = min(8, os.cpu_count() or 1, cfg.H)
+    if n > 1:
+        with mp.get_context("spawn").Pool(n) as pool:
+            parts = pool.map(_gen_head, [(cfg.name, h) for h in range(cfg.H)])
+    else:
+        parts = [_gen_head((cfg.name, h)) for h in range(cfg.H)]
+    return [np.stack([p[i] for p in parts]) for i in range(5)]
+
+
+class Clocks:
+    """nvidia-smi sampling of SM clocks and throttle reasons over a region."""
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_id):
+        self.gpu_id = gpu_id
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        try:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu_id), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200", "-f", self.path],
+                stdout=subprocess.DEVNULL, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self):
+        if not self.path or not os.path.exists(self.path):
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"]}
+        rows = []
+        for line in open(self.path):
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 8:
+                continue
+            try:
+                rows.append((float(f[0]), float(f[1]), f[4], f[5], f[6], f[7]))
+            except ValueError:
+                continue
+        os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+        reasons = sorted({n for r in rows for n, v in zip(names, r[2:]) if v.lower() == "active"})
+        return {"sm_mhz": statistics.median(r[0] for r in rows), "sm_max_mhz": max(r[1] for r in rows),
+                "reasons": reasons, "samples": len(rows)}
+
+
+def _peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            p = json.load(f)
+        return p["bf16_tflops_sustained"], p["hbm_gbs"], "measured"
+    except Exception:
+        return 1400.0, 6650.0, "fallback"
+
+
+# ----------------------------------------------------------------- oracle
+
+def oracle_sample(cfg, rho, q, k, v, iq, ik):
+    """Time the CPU oracle on a bounded sample of one head and extrapolate to
+    the whole layer.  Returns (seconds per layer, description, threads)."""
+    import numpy as np
+    from oracle import svgear_oracle as ora
+    s = 1.0 / math.sqrt(cfg.d)
+    t = {}
+    t0 = time.perf_counter()
+    lab_q = ora.assign(q, iq); mu_q, _ = ora.update(q, lab_q, iq)
+    t["kmeans_q_iter"] = time.perf_counter() - t0
+    t0 = time.perf_counter()
+    lab_k = ora.assign(k, ik); mu_k, _ = ora.update(k, lab_k, ik)
+    t["kmeans_k_iter"] = time.perf_counter() - t0
+    t0 = time.perf_counter()
+    lq = ora.assign(q, mu_q); lk = ora.assign(k, mu_k)
+    t["final_assign"] = time.perf_counter() - t0
+    t0 = time.perf_counter()
+    pq, oq, cq = ora.permute(lq, cfg.Cq); pk, ok, ck = ora.permute(lk, cfg.Ck)
+    Vbar = ora.value_centroids(v, lk, cfg.Ck)
+    _ = (q[pq], k[pk], v[pk])
+    t["permute"] = time.perf_counter() - t0
+    frac = 8
+    sub = slice(0, cfg.N // frac)
+    t0 = time.perf_counter()
+    E_part, M = ora.block_error(mu_q, mu_k, Vbar, k[sub], v[sub], lk[sub], ck, s)
+    t["block_error"] = (time.perf_counter() - t0) * frac
+    E = E_part
+    t0 = time.perf_counter()
+    mask, _, _ = ora.route(E, ck, cq, rho)
+    t["route"] = time.perf_counter() - t0
+    rows = np.nonzero(np.isin(lq, np.arange(min(4, cfg.Cq))))[0][:512]
+    lq_s = np.full_like(lq, -1)
+    lq_s[rows] = lq[rows]
+    t0 = time.perf_counter()
+    ora.hybrid_attention(q, k, v, lq_s, lk, mu_k, Vbar, ck, mask, s)
+    t["attn"] = (time.perf_counter() - t0) * (cfg.N / max(1, rows.size))
+    per_head = (cfg.iters * (t["kmeans_q_iter"] + t["kmeans_k_iter"]) + t["final_assign"]
+                + t["permute"] + t["block_error"] + t["route"] + t["attn"])
+    desc = (f"oracle (float64 NumPy) on head 0: one k-means round of Q and K timed and x{cfg.iters}, "
+            f"final assignment, permutation, block error on 1/{frac} of the keys (x{frac}), routing, "
+            f"hybrid attention on {rows.size} query rows (x N/rows); extrapolated to {cfg.H} heads")
+    return per_head * cfg.H, desc, t
+
+
+def _threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads") for i in threadpool_info() if i.get("user_api") == "blas"]
+        return int(max(n)) if n else (os.cpu_count() or 1)
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def dense_flops(cfg):
+    return 4.0 * cfg.H * cfg.N * cfg.N * cfg.d
+
+
+def run_reference(a, cfg, rho):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    import numpy as np
+    from clustered_sparse_attention_flash_b200 import synth
+    q, k, v, _ = synth.make_head(cfg, 0)
+    iq = synth.forgy_init(cfg, q, 0, 0, cfg.Cq)
+    ik = synth.forgy_init(cfg, k, 0, 1, cfg.Ck)
+    secs = []
+    for i in range(a.warmup + a.steps):
+        t0 = time.perf_counter()
+        est, desc, _ = oracle_sample(cfg, rho, q, k, v, iq, ik)
+        if i >= a.warmup:
+            secs.append(est)
+    layer_s = statistics.mean(secs)
+    val = dense_flops(cfg) / layer_s / 1e12
+    line = {"impl": "reference", "metric": METRIC, "value": val, "unit": UNIT, "n_gpus": a.gpus,
+            "steps": a.steps, "warmup": a.warmup, "ms_per_step": layer_s * 1e3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": {"workload": _workload(cfg, rho)},
+            "cpu_baseline": {"value": val, "unit": UNIT, "cores": _threads(), "kind": "oracle",
+                             "sample": desc},
+            "e2e": {"value": val, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# -------------------------------------------------------------------- ours
+
+def main():
+    a = _args()
+    from clustered_sparse_attention_flash_b200 import synth
+    cfg = synth.CONFIGS[a.config]
+    rho = cfg.rho if a.rho is None else a.rho
+    if a.impl == "reference":
+        return run_reference(a, cfg, rho)
+    assert a.warmup >= 3, "at least 3 warm-up steps"
+
+    q_np, k_np, v_np, iq_np, ik_np = generate(cfg)   # before any CUDA call
+
+    import numpy as np
+    import torch
+    from clustered_sparse_attention_flash_b200 import svgear as sv
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dist = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=600))
+    dev = torch.device("cuda", local)
+    tdt = torch.bfloat16 if cfg.dtype == "bf16" else torch.float32
+    Q = torch.from_numpy(q_np).to(tdt).pin_memory()
+    K = torch.from_numpy(k_np).to(tdt).pin_memory()
+    V = torch.from_numpy(v_np).to(tdt).pin_memory()
+    dQ, dK, dV = Q.to(dev), K.to(dev), V.to(dev)
+    iq, ik = torch.from_numpy(iq_np).to(dev), torch.from_numpy(ik_np).to(dev)
+    dO = torch.empty_like(dQ)
+    hO = torch.empty_like(Q).pin_memory()
+    s = 1.0 / math.sqrt(cfg.d)
+    p = sv.params(cfg.H, cfg.N, cfg.N, cfg.d, cfg.Cq, cfg.Ck, cfg.iters, rho, s,
+                  sv.SVGEAR_BF16 if cfg.dtype == "bf16" else sv.SVGEAR_F32)
+    ws = sv.workspace(sv.svgear_workspace_size(p), dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        sv.svgear_forward(dQ, dK, dV, p, iq, ik, dO, ws, ws.numel(), stream)
+
+    def barrier():
+        if dist is not None:
+            dist.barrier()
+
+    for _ in range(a.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    assert sv.svgear_get_status(stream) == sv.SVGEAR_OK
+
+    # ---- timed region: K steps on inputs resident in HBM
+    props = torch.cuda.get_device_properties(dev)
+    gpu_id = getattr(props, "uuid", None)
+    gpu_id = f"GPU-{gpu_id}" if gpu_id is not None and not str(gpu_id).startswith("GPU-") else (gpu_id or local)
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier()
+    torch.cuda.synchronize(dev)
+    l0 = sv.svgear_launch_count()
+    with Clocks(gpu_id) as clk:
+        ev0.record(stream)
+        for _ in range(a.steps):
+            step()
+        ev1.record(stream)
+        torch.cuda.synchronize(dev)
+    launches = sv.svgear_launch_count() - l0
+    barrier()
+    ms = ev0.elapsed_time(ev1) / a.steps
+    if dist is not None:
+        t = torch.tensor([ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    clocks = clk.summary()
+
+    # ---- per-stage breakdown (library-internal CUDA events on the same stream)
+    stats = []
+    for _ in range(a.steps):
+        st = sv.svgear_stats()
+        sv.svgear_forward(dQ, dK, dV, p, iq, ik, dO, ws, ws.numel(), stream, st)
+        stats.append(st.as_dict())
+    avg = {k2: statistics.mean(x[k2] for x in stats) for k2 in stats[0]}
+    exec_pairs, comp_pairs = avg["exec_pairs"], avg["comp_pairs"]
+    routing_ms = avg["ms_kmeans_q"] + avg["ms_kmeans_k"] + avg["ms_permute"] + avg["ms_block_error"] + avg["ms_route"]
+
+    # ---- end to end: pinned host buffers in, result back to host, every step
+    e2e = None
+    if not a.no_e2e:
+        for _ in range(1):
+            dQ.copy_(Q, non_blocking=True); dK.copy_(K, non_blocking=True); dV.copy_(V, non_blocking=True)
+            step(); hO.copy_(dO, non_blocking=True)
+        barrier()
+        torch.cuda.synchronize(dev)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(a.steps):
+            dQ.copy_(Q, non_blocking=True); dK.copy_(K, non_blocking=True); dV.copy_(V, non_blocking=True)
+            step()
+            hO.copy_(dO, non_blocking=True)
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        ems = e0.elapsed_time(e1) / a.steps
+        if dist is not None:
+            t = torch.tensor([ems], device=dev)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            ems = float(t.item())
+        bi = 3 * Q.numel() * Q.element_size()
+        bo = hO.numel() * hO.element_size()
+        e2e = {"value": world * dense_flops(cfg) / (ems / 1e3) / 1e12, "unit": UNIT,
+               "h2d_bytes_per_step": bi, "d2h_bytes_per_step": bo, "ms_per_step": ems}
+
+    peak_tc, peak_hbm, peak_src = _peaks()
+    attn_flops = 4.0 * cfg.d * (exec_pairs + comp_pairs)
+    achieved = attn_flops / (avg["ms_attn"] / 1e3) / 1e12
+    roofline = {"kernel": "hybrid attention (svgear_hybrid_attn)", "bound": "tensor",
+                "achieved": achieved, "peak": peak_tc, "unit": "TFLOP/s", "frac": achieved / peak_tc,
+                "traffic": None,
+                "note": f"algorithmic 4*d*(executed + compensated pairs) per launch over the stage's "
+                        f"CUDA-event time; peak = {peak_src} sustained dense bf16"}
+
+    cpu = None
+    if rank == 0 and world == 1 and not a.no_cpu_baseline:
+        sec, desc, _ = oracle_sample(cfg, rho, q_np[0], k_np[0], v_np[0], iq_np[0], ik_np[0])
+        cpu = {"value": dense_flops(cfg) / sec / 1e12, "unit": UNIT, "cores": _threads(),
+               "kind": "oracle", "sample": desc, "layer_s_extrapolated": sec}
+
+    value = world * dense_flops(cfg) / (ms / 1e3) / 1e12
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": a.steps,
+        "warmup": a.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": cfg.dtype, "data": "synthetic",
+        "config": {"workload": _workload(cfg, rho),
+                   "l2": "inputs (3 x %.2f GB) larger than the 126 MB L2; no flush" % (Q.numel() * Q.element_size() / 1e9),
+                   "parallelism": f"replicas x{world} (heads independent; no data-path collective)"},
+        "layer_ms": ms,
+        "exec_pair_tflops": 4.0 * cfg.d * exec_pairs / (avg["ms_attn"] / 1e3) / 1e12,
+        "exec_pair_frac_of_peak": (4.0 * cfg.d * exec_pairs / (avg["ms_attn"] / 1e3) / 1e12) / peak_tc,
+        "routing_overhead_pct": 100.0 * routing_ms / avg["ms_total"],
+        "routing_overhead_excl_kmeans_pct": 100.0 * (avg["ms_permute"] + avg["ms_block_error"] + avg["ms_route"]) / avg["ms_total"],
+        "stage_ms": {k2: avg[k2] for k2 in ("ms_kmeans_q", "ms_kmeans_k", "ms_permute", "ms_block_error",
+                                            "ms_route", "ms_attn", "ms_total")},
+        "density": exec_pairs / (cfg.H * cfg.N * cfg.N),
+        "roofline": roofline,
+        "cpu_baseline": cpu,
+        "e2e": e2e,
+        "gpu_launches": launches,
+        "gpu_launches_per_step": launches / a.steps,
+        "clocks": clocks,
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,154 @@
+// Value-aware block error with the query-centroid proxy (SVG-EAR review,
+// step (2); gist.science summary 2.B, "lightweight probe", O(C_q N_k d)).
+//
+//   eps^2(a,j) = || A vbar_c - B_j v_j ||^2,  A = e^{s qbar_a.kbar_c - M_a},
+//                                              B_j = e^{s qbar_a.k_j - M_a}
+//   E[a,c]     = (1/|k_c|) sum_{j in c} eps^2(a,j)
+//
+// The norm is expanded with per-key terms precomputed by the permute step
+// (s1 = ||vbar-v||^2, s2 = (vbar-v).v, s3 = ||v||^2) around A:
+//   A vbar - B v = A (vbar - v) + (A - B) v,  A - B = -A expm1(u),
+//   u = s qbar_a.(k_j - kbar_c),
+//   eps^2 = A^2 s1 + 2 A (A-B) s2 + (A-B)^2 s3.
+// This is exact algebra; the form keeps full relative accuracy when the
+// cluster is tight (u -> 0, v -> vbar) where a^2|vbar|^2 - 2ab vbar.v + b^2|v|^2
+// would cancel.  Logits never leave registers.
+#include "common.cuh"
+#include "internal.h"
+
+namespace svg {
+
+namespace {
+
+// L[a][c] = s qbar_a.kbar_c (float64 dot, stored float32) and
+// M[a] = max over non-empty c of L[a][c].  One block per (a, head).
+template <int D>
+__global__ void __launch_bounds__(256) k_centroid_logits(const float* __restrict__ Qbar,
+                                                         const float* __restrict__ Kbar,
+                                                         const int32_t* __restrict__ k_off, int Cq,
+                                                         int Ck, float scale, float* __restrict__ L,
+                                                         float* __restrict__ M) {
+  __shared__ float q[D];
+  __shared__ float red[32];
+  const int h = blockIdx.y, a = blockIdx.x;
+  for (int t = threadIdx.x; t < D; t += blockDim.x) q[t] = Qbar[((size_t)h * Cq + a) * D + t];
+  __syncthreads();
+  const int32_t* off = k_off + (size_t)h * (Ck + 1);
+  float mx = -INFINITY;
+  for (int c = threadIdx.x; c < Ck; c += blockDim.x) {
+    const float* kb = Kbar + ((size_t)h * Ck + c) * D;
+    double acc = 0.0;
+#pragma unroll 8
+    for (int t = 0; t < D; ++t) acc = fma((double)q[t], (double)kb[t], acc);
+    const float l = (float)(acc * (double)scale);
+    L[((size_t)h * Cq + a) * Ck + c] = l;
+    if (off[c + 1] > off[c]) mx = fmaxf(mx, l);
+  }
+  for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = mx;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    float m = -INFINITY;
+    for (int w = 0; w < (int)(blockDim.x >> 5); ++w) m = fmaxf(m, red[w]);
+    M[(size_t)h * Cq + a] = m;
+  }
+}
+
+// One block per (key cluster c, head); thread t owns query cluster a = t (+128k).
+// Keys of c stream through shared memory as k_j - kbar_c.
+template <typename T, int D>
+__global__ void __launch_bounds__(128) k_block_error(const float* __restrict__ Qbar,
+                                                     const float* __restrict__ Kbar,
+                                                     const T* __restrict__ Kp,
+                                                     const int32_t* __restrict__ k_off,
+                                                     const float* __restrict__ ks, const float* __restrict__ L,
+                                                     const float* __restrict__ M, int H, int Nk, int Cq,
+                                                     int Ck, float scale, float* __restrict__ E) {
+  constexpr int KT = 32;
+  __shared__ __align__(16) float dk[KT][D];
+  __shared__ float sc[3][KT];
+  __shared__ float kb[D];
+  const int h = blockIdx.y, c = blockIdx.x;
+  const int beg = k_off[(size_t)h * (Ck + 1) + c], end = k_off[(size_t)h * (Ck + 1) + c + 1];
+  if (beg >= end) {
+    for (int a = threadIdx.x; a < Cq; a += blockDim.x) E[((size_t)h * Cq + a) * Ck + c] = 0.f;
+    return;
+  }
+  for (int t = threadIdx.x; t < D; t += blockDim.x) kb[t] = Kbar[((size_t)h * Ck + c) * D + t];
+  const size_t plane = (size_t)H * Nk;
+  const T* Kh = Kp + (size_t)h * Nk * D;
+  for (int a0 = 0; a0 < Cq; a0 += blockDim.x) {
+    const int a = a0 + threadIdx.x;
+    const bool act = a < Cq;
+    float q[D];
+    float A = 0.f;
+    if (act) {
+      const float* qb = Qbar + ((size_t)h * Cq + a) * D;
+#pragma unroll
+      for (int t = 0; t < D; t += 4) {
+        float4 v = ld4(qb + t);
+        q[t] = v.x * scale; q[t + 1] = v.y * scale; q[t + 2] = v.z * scale; q[t + 3] = v.w * scale;
+      }
+      A = expf(L[((size_t)h * Cq + a) * Ck + c] - M[(size_t)h * Cq + a]);
+    } else {
+#pragma unroll
+      for (int t = 0; t < D; ++t) q[t] = 0.f;
+    }
+    double acc = 0.0;
+    for (int j0 = beg; j0 < end; j0 += KT) {
+      const int nk = min(KT, end - j0);
+      __syncthreads();
+      for (int e = threadIdx.x; e < nk * D; e += blockDim.x) {
+        const int r = e / D, t = e % D;
+        dk[r][t] = to_f(Kh[(size_t)(j0 + r) * D + t]) - kb[t];
+      }
+      for (int e = threadIdx.x; e < 3 * nk; e += blockDim.x) {
+        const int w = e / nk, r = e % nk;
+        sc[w][r] = ks[w * plane + (size_t)h * Nk + j0 + r];
+      }
+      __syncthreads();
+      if (act) {
+        for (int r = 0; r < nk; ++r) {
+          float u = 0.f;
+#pragma unroll
+          for (int t = 0; t < D; t += 4) {
+            const float4 k4 = *reinterpret_cast<const float4*>(&dk[r][t]);
+            u = fmaf(q[t], k4.x, u); u = fmaf(q[t + 1], k4.y, u);
+            u = fmaf(q[t + 2], k4.z, u); u = fmaf(q[t + 3], k4.w, u);
+          }
+          const float amb = -A * expm1f(u);
+          float e2 = A * A * sc[0][r] + 2.f * A * amb * sc[1][r] + amb * amb * sc[2][r];
+          acc += (double)fmaxf(e2, 0.f);
+        }
+      }
+    }
+    if (act) E[((size_t)h * Cq + a) * Ck + c] = (float)(acc / (double)(end - beg));
+  }
+}
+
+}  // namespace
+
+size_t block_error_ws_bytes(int H, int Cq, int Ck) {
+  return align_up((size_t)H * Cq * Ck * sizeof(float), 256);
+}
+
+cudaError_t block_error_run(const float* Qbar, const float* Kbar, const float* Vbar,
+                            const void* Kp, const void* Vp, const int32_t* k_off,
+                            const float* key_scalars, int dtype, int H, int Nk, int d, int Cq,
+                            int Ck, float scale, float* E, float* M, void* ws, cudaStream_t st) {
+  (void)Vbar; (void)Vp;  // their contribution enters through key_scalars
+  float* L = static_cast<float*>(ws);
+  if (d == 128) { k_centroid_logits<128><<<dim3(Cq, H), 256, 0, st>>>(Qbar, Kbar, k_off, Cq, Ck, scale, L, M); note_launch(); }
+  else { k_centroid_logits<64><<<dim3(Cq, H), 256, 0, st>>>(Qbar, Kbar, k_off, Cq, Ck, scale, L, M); note_launch(); }
+  dim3 g(Ck, H);
+  if (dtype == DT_BF16) {
+    if (d == 128) { k_block_error<bf16, 128><<<g, 128, 0, st>>>(Qbar, Kbar, static_cast<const bf16*>(Kp), k_off, key_scalars, L, M, H, Nk, Cq, Ck, scale, E); note_launch(); }
+    else { k_block_error<bf16, 64><<<g, 128, 0, st>>>(Qbar, Kbar, static_cast<const bf16*>(Kp), k_off, key_scalars, L, M, H, Nk, Cq, Ck, scale, E); note_launch(); }
+  } else {
+    if (d == 128) { k_block_error<float, 128><<<g, 128, 0, st>>>(Qbar, Kbar, static_cast<const float*>(Kp), k_off, key_scalars, L, M, H, Nk, Cq, Ck, scale, E); note_launch(); }
+    else { k_block_error<float, 64><<<g, 128, 0, st>>>(Qbar, Kbar, static_cast<const float*>(Kp), k_off, key_scalars, L, M, H, Nk, Cq, Ck, scale, E); note_launch(); }
+  }
+  return cudaGetLastError();
+}
+
+}  // namespace svg

@@ -1,0 +1,72 @@
+// Host-side launchers shared between the translation units of libsvgear.so.
+// Every launcher only enqueues on `st` and returns cudaGetLastError().
+#pragma once
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+namespace svg {
+
+// Device status word of the current device (see svgear_get_status).
+int* status_word();
+
+// Counts kernel launches issued by the library (svgear_launch_count).
+void note_launch();
+
+// ---- stable counting sort of labels (shared by k-means update and permute)
+// chunk = tokens per scatter chunk; nchunk = ceil(N / chunk)
+constexpr int kSortChunk = 512;
+size_t sort_ws_bytes(int H, int N, int C);
+// Fills counts [H,C], offsets [H,C+1] and (if perm != null) perm [H,N].
+cudaError_t cluster_sort(const int32_t* labels, int H, int N, int C, int32_t* counts,
+                         int32_t* offsets, int32_t* perm, void* ws, cudaStream_t st);
+
+// ---- k-means
+size_t kmeans_ws_bytes(int H, int N, int d, int C);
+cudaError_t kmeans_run(const void* X, int dtype, int H, int N, int d, int C, int iters,
+                       const float* init, float* cent, int32_t* labels, int32_t* counts,
+                       int32_t* offsets_out, int32_t* perm_out, void* ws, cudaStream_t st);
+
+// ---- permute / value centroids / per-key scalars
+cudaError_t gather_rows(const void* X, int dtype, const int32_t* perm, int H, int N, int d,
+                        void* Xp, cudaStream_t st);
+cudaError_t value_stats(const void* Vp, int dtype, const int32_t* off, int H, int N, int d,
+                        int C, float* Vbar, float* key_scalars, cudaStream_t st);
+
+// ---- block error
+size_t block_error_ws_bytes(int H, int Cq, int Ck);
+cudaError_t block_error_run(const float* Qbar, const float* Kbar, const float* Vbar,
+                            const void* Kp, const void* Vp, const int32_t* k_off,
+                            const float* key_scalars, int dtype, int H, int Nk, int d, int Cq,
+                            int Ck, float scale, float* E, float* M, void* ws, cudaStream_t st);
+
+// ---- routing
+cudaError_t route_run(const float* E, const int32_t* k_counts, const int32_t* q_counts,
+                      int H, int Nk, int Cq, int Ck, float rho, uint8_t* mask, int32_t* sel,
+                      int32_t* n_sel, int64_t* exec_pairs, cudaStream_t st);
+
+// ---- hybrid attention
+size_t attn_ws_bytes(int H, int Nq, int d, int Cq, int Ck);
+cudaError_t attn_run(const void* Qp, const void* Kp, const void* Vp, const int32_t* q_off,
+                     const int32_t* k_off, const int32_t* perm_q, const float* Kbar,
+                     const float* Vbar, const int32_t* sel, const int32_t* n_sel, int dtype,
+                     int H, int Nq, int Nk, int d, int Cq, int Ck, float scale, void* O,
+                     void* ws, cudaStream_t st);
+
+inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+// Bump allocator over a caller-provided workspace.
+struct Carve {
+  char* base;
+  size_t off = 0;
+  explicit Carve(void* p) : base(static_cast<char*>(p)) {}
+  template <typename T> T* take(size_t n) {
+    off = align_up(off, 256);
+    T* p = base ? reinterpret_cast<T*>(base + off) : nullptr;
+    off += n * sizeof(T);
+    return p;
+  }
+  size_t used() const { return align_up(off, 256); }
+};
+
+}  // namespace svg

@@ -1,0 +1,224 @@
+/*
+ * svgear.h -- C ABI of libsvgear.so, the B200 (sm_100a) SVG-EAR sparse-attention
+ * operator.
+ *
+ * The operator is the inference pipeline of "SVG-EAR: Parameter-Free Linear
+ * Compensation for Sparse Video Generation via Error-aware Routing"
+ * (arXiv 2603.08982), as summarised by the paper.rainbus.top review
+ * ("complete inference pipeline", steps (1)-(5)) and the gist.science technical
+ * summaries (sections 2.A-2.C):
+ *   (1) semantic k-means of queries and keys, tokens reordered so that every
+ *       cluster is contiguous                         -> svgear_kmeans, svgear_permute
+ *   (2) value-aware block error with the query-centroid proxy
+ *                                                     -> svgear_block_error
+ *   (3) error-to-cost greedy routing under the density budget rho
+ *                                                     -> svgear_route
+ *   (4) hybrid attention: exact softmax attention on routed blocks, centroid
+ *       linear compensation on the rest, one joint softmax
+ *                                                     -> svgear_hybrid_attn
+ *   all of it on one stream                           -> svgear_forward
+ *
+ * Conventions (every entry point):
+ *  - Tensor pointers are DEVICE pointers owned by the caller.  The library
+ *    never allocates device memory; scratch comes from a caller-provided
+ *    workspace whose size the matching *_workspace_size call returns.
+ *  - Tensors are dense and row-major, per head h: X[h][n][t] at
+ *    X + (h*N + n)*d + t.  Rows must be 16-byte aligned (d in {64, 128}).
+ *    Element type of Q/K/V-like tensors is `dtype` (float32 or bfloat16);
+ *    centroids, errors and per-key scalars are float32; indices int32.
+ *  - `stream` is a cudaStream_t (NULL = legacy default stream); every call only
+ *    enqueues work and returns.  Calls on one stream run in order.
+ *  - The return value reports host-side validation and launch errors only
+ *    (svgear_status).  Nothing is enqueued when validation fails.  Faults
+ *    and timed-out waits inside kernels are recorded in a device status word
+ *    that svgear_get_status reads.
+ *  - No exceptions or aborts cross the ABI.
+ */
+#ifndef SVGEAR_H
+#define SVGEAR_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define SVGEAR_API __attribute__((visibility("default")))
+#else
+#define SVGEAR_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  SVGEAR_OK = 0,
+  SVGEAR_ERR_INVALID = -1,     /* bad argument (null pointer, size, range) */
+  SVGEAR_ERR_UNSUPPORTED = -2, /* valid but not implemented (d, dtype) */
+  SVGEAR_ERR_CUDA = -3,        /* a CUDA runtime call or launch failed */
+  SVGEAR_ERR_TIMEOUT = -4,     /* a bounded in-kernel wait gave up */
+  SVGEAR_ERR_WORKSPACE = -5    /* workspace missing or too small */
+} svgear_status;
+
+typedef enum { SVGEAR_F32 = 0, SVGEAR_BF16 = 1 } svgear_dtype;
+
+/* Operator hyper-parameters of one attention layer. */
+typedef struct {
+  int H;        /* heads (independent problems) */
+  int Nq, Nk;   /* query / key tokens per head */
+  int d;        /* head dimension: 64 or 128 */
+  int Cq, Ck;   /* query / key clusters, 1 <= C <= N */
+  int iters;    /* k-means assign->update rounds (>= 0) */
+  float rho;    /* density budget in [0, 1]: each query cluster computes at
+                   most floor(rho * Nk) keys exactly */
+  float scale;  /* softmax scale; <= 0 selects 1/sqrt(d) */
+  int dtype;    /* svgear_dtype of Q, K, V and the output */
+} svgear_params;
+
+/* Per-stage device times of one svgear_forward call (CUDA events). */
+typedef struct {
+  float ms_kmeans_q, ms_kmeans_k, ms_permute, ms_block_error, ms_route, ms_attn;
+  float ms_total;
+  int64_t exec_pairs;   /* sum over heads of sum_a |q_a| * sum_{c routed} |k_c| */
+  int64_t comp_pairs;   /* sum over heads of sum_a |q_a| * #compensated non-empty c */
+} svgear_stats;
+
+/* Device pointers to the intermediates svgear_forward leaves in its workspace. */
+typedef struct {
+  float *cent_q, *cent_k;          /* [H,Cq,d], [H,Ck,d] k-means centroids */
+  float *vbar;                     /* [H,Ck,d] value centroids */
+  int32_t *labels_q, *labels_k;    /* [H,Nq], [H,Nk] */
+  int32_t *counts_q, *counts_k;    /* [H,Cq], [H,Ck] */
+  int32_t *perm_q, *perm_k;        /* [H,Nq], [H,Nk]: perm[new] = old */
+  int32_t *off_q, *off_k;          /* [H,Cq+1], [H,Ck+1] */
+  void *Qp, *Kp, *Vp;              /* permuted copies, dtype */
+  float *key_scalars;              /* [3,H,Nk] */
+  float *E, *M;                    /* [H,Cq,Ck], [H,Cq] */
+  uint8_t *mask;                   /* [H,Cq,Ck] */
+  int32_t *sel, *n_sel;            /* [H,Cq,Ck], [H,Cq] */
+  int64_t *exec_pairs;             /* [H] */
+} svgear_views;
+
+/* Library version string (static storage). */
+SVGEAR_API const char* svgear_version(void);
+
+/* Number of CUDA kernels this library has launched in this process (all
+ * devices, all streams); a host-side counter, no device access. */
+SVGEAR_API long long svgear_launch_count(void);
+
+/* Human-readable text of a status code (static storage, never NULL). */
+SVGEAR_API const char* svgear_status_string(int status);
+
+/* Synchronises `stream`, then returns and clears the device status word of the
+ * current device: SVGEAR_OK, or SVGEAR_ERR_TIMEOUT when a bounded in-kernel
+ * wait expired since the last call; SVGEAR_ERR_CUDA if the synchronisation
+ * itself failed (a sticky CUDA error). */
+SVGEAR_API int svgear_get_status(void* stream);
+
+/* ---------------------------------------------------------------------------
+ * (1) k-means (Lloyd) on X [H,N,d] with C clusters.  Review step (1), "Flash
+ * k-means" clustering of queries and keys; gist.science summary 2.A.
+ *   init    [H,C,d] float32 initial centroid values; NULL selects the
+ *           deterministic init mu_c = x_{floor(c*N/C)}.
+ *   cent    [H,C,d] float32 out: centroids after `iters` rounds of
+ *           assign->update (an empty cluster keeps its previous centroid).
+ *   labels  [H,N] int32 out: argmin_c ||x - mu_c||^2 against the final
+ *           centroids (ties -> smaller index).
+ *   counts  [H,C] int32 out: cluster sizes of `labels`.
+ *   ws      device scratch of at least svgear_kmeans_workspace_size bytes.
+ * Labels are exact: near-ties of the float32 tensor-core scores are re-decided
+ * in float64.  Centroid sums are deterministic (no float atomics).
+ * ------------------------------------------------------------------------- */
+SVGEAR_API size_t svgear_kmeans_workspace_size(int H, int N, int d, int C);
+SVGEAR_API int svgear_kmeans(const void* X, int dtype, int H, int N, int d, int C, int iters,
+                  const float* init, float* cent, int32_t* labels, int32_t* counts,
+                  void* ws, size_t ws_bytes, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * (1') Reorder tokens so that each cluster is contiguous.  Review step (1).
+ * Stable counting sort by label: perm[h][new] = old, clusters in index
+ * order, original order inside a cluster; offsets [H,C+1] exclusive prefix
+ * of the cluster sizes.  Xp[h][new] = X[h][perm[h][new]].
+ * When V is non-NULL (the keys' values, same N), also
+ *   Vp      [H,N,d] values gathered with the same perm,
+ *   Vbar    [H,C,d] float32 mean of v over each cluster (0 if empty),
+ *   key_scalars [3,H,N] float32 in permuted order: ||vbar_c - v_j||^2,
+ *           (vbar_c - v_j).v_j, ||v_j||^2 -- the per-key terms of the
+ *           value-aware error expansion.  Vbar / key_scalars may be NULL.
+ * ------------------------------------------------------------------------- */
+SVGEAR_API size_t svgear_permute_workspace_size(int H, int N, int C);
+SVGEAR_API int svgear_permute(const void* X, int dtype, const int32_t* labels, int H, int N,
+                   int d, int C, void* Xp, int32_t* perm, int32_t* offsets,
+                   const void* V, void* Vp, float* Vbar, float* key_scalars,
+                   void* ws, size_t ws_bytes, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * (2) Value-aware block error with the query-centroid proxy.  Review step (2);
+ * gist.science 2.B ("lightweight probe", O(C_q N_k d)).  For query cluster a
+ * and key cluster c (keys j of c, s = scale):
+ *   eps^2(a,j) = || exp(s qbar_a.kbar_c) vbar_c - exp(s qbar_a.k_j) v_j ||^2
+ *   E[h][a][c] = exp(-2 M_a) * (1/|k_c|) * sum_{j in c} eps^2(a,j)
+ *   M[h][a]    = max over non-empty c of s qbar_a.kbar_c
+ * E is the pages' error-to-cost ratio times the positive per-row factor
+ * exp(-2 M_a), which keeps it in float32 range and leaves the routing order
+ * unchanged.  Empty key clusters get E = 0.
+ *   Qbar [H,Cq,d], Kbar/Vbar [H,Ck,d] float32; Kp/Vp [H,Nk,d] dtype (keys in
+ *   cluster order); k_off [H,Ck+1]; key_scalars [3,H,Nk] from svgear_permute.
+ * ------------------------------------------------------------------------- */
+SVGEAR_API size_t svgear_block_error_workspace_size(const svgear_params* p);
+SVGEAR_API int svgear_block_error(const float* Qbar, const float* Kbar, const float* Vbar,
+                       const void* Kp, const void* Vp, const int32_t* k_off,
+                       const float* key_scalars, const svgear_params* p,
+                       float* E, float* M, void* ws, size_t ws_bytes, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * (3) Error-aware routing.  Review step (3); gist.science 2.B "Selektion".
+ * Per (h, a): non-empty key clusters in E-descending order (equal E: smaller
+ * c first); the longest prefix whose total size fits floor(rho*Nk) is routed
+ * to exact attention.
+ *   mask [H,Cq,Ck] uint8 out (1 = exact), sel [H,Cq,Ck] int32 out (routed
+ *   clusters in routing order, first n_sel[h][a] valid), n_sel [H,Cq] out,
+ *   exec_pairs [H] int64 out (sum_a |q_a| * sum_{c routed} |k_c|).
+ *   k_counts [H,Ck], q_counts [H,Cq] int32.  Ck <= 4096.
+ * ------------------------------------------------------------------------- */
+SVGEAR_API int svgear_route(const float* E, const int32_t* k_counts, const int32_t* q_counts,
+                 const svgear_params* p, uint8_t* mask, int32_t* sel, int32_t* n_sel,
+                 int64_t* exec_pairs, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * (4) Hybrid attention.  Review step (4); gist.science 2.A "lineare
+ * Kompensation".  For query i of cluster a (permuted order):
+ *   o_i = sum over routed c, j in c of e^{s q_i.k_j} v_j
+ *         + sum over compensated non-empty c of |k_c| e^{s q_i.kbar_c} vbar_c
+ *         divided by the same sums without v  (one max, one normaliser)
+ * and o_i is written to O[h][perm_q[h][i]] (original token order).
+ *   Qp [H,Nq,d], Kp/Vp [H,Nk,d] dtype; q_off [H,Cq+1], k_off [H,Ck+1];
+ *   Kbar/Vbar [H,Ck,d] float32; sel/n_sel from svgear_route; O [H,Nq,d] dtype.
+ * ------------------------------------------------------------------------- */
+SVGEAR_API size_t svgear_hybrid_attn_workspace_size(const svgear_params* p);
+SVGEAR_API int svgear_hybrid_attn(const void* Qp, const void* Kp, const void* Vp,
+                       const int32_t* q_off, const int32_t* k_off, const int32_t* perm_q,
+                       const float* Kbar, const float* Vbar, const int32_t* sel,
+                       const int32_t* n_sel, const svgear_params* p, void* O,
+                       void* ws, size_t ws_bytes, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * The whole operator: (1) -> (1') -> (2) -> (3) -> (4) on one stream.
+ *   Q [H,Nq,d], K/V [H,Nk,d], O [H,Nq,d] in `dtype`.
+ *   init_q [H,Cq,d] / init_k [H,Ck,d] float32 k-means initial centroids
+ *   (NULL: deterministic init, see svgear_kmeans).
+ *   ws: at least svgear_workspace_size(p) bytes; holds every intermediate
+ *   (svgear_forward_views locates them).
+ *   stats: NULL, or filled with per-stage device times -- then the call
+ *   records CUDA events and synchronises `stream` before returning.
+ * ------------------------------------------------------------------------- */
+SVGEAR_API size_t svgear_workspace_size(const svgear_params* p);
+SVGEAR_API int svgear_forward_views(const svgear_params* p, void* ws, size_t ws_bytes,
+                         svgear_views* out);
+SVGEAR_API int svgear_forward(const void* Q, const void* K, const void* V, const svgear_params* p,
+                   const float* init_q, const float* init_k, void* O, void* ws,
+                   size_t ws_bytes, void* stream, svgear_stats* stats);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* SVGEAR_H */
