@@ -322,3 +322,24 @@ def test_forward_empty_key_cluster():
     assert host(views["mask"])[0, :, 5].sum() == 0
     o = ora.forward(q[0], k[0], v[0], 4, 6, 3, 0.4, s, iq[0], ik[0])
     assert_close(host(O)[0], o["O"], *OUT_TOL["f32"], "empty-cluster output")
+
+
+# ------------------------------------- tensor-core assignment, wide shapes
+
+@pytest.mark.parametrize("N,d,C,seed", [
+    (75600, 128, 500, 0),    # Wan-shaped key clustering: two accumulator slots
+    (20000, 128, 300, 1),    # second slot ends in a 16-column tail
+    (9001, 64, 1000, 2),     # d = 64: four slots alternate between warpgroups
+    (5000, 128, 100, 3),     # one slot, tiles alternate between warpgroups
+])
+def test_kmeans_assign_wide(N, d, C, seed):
+    from clustered_sparse_attention_flash_b200.synth import to_bf16_f32
+    rng = np.random.default_rng(seed)
+    centers = rng.standard_normal((C // 2, d)).astype(np.float32) * 1.3
+    X = to_bf16_f32(centers[rng.integers(0, C // 2, N)] + 0.5 * rng.standard_normal((N, d)).astype(np.float32))
+    mu = X[rng.choice(N, C, replace=False)].astype(np.float32)
+    mu = (mu + 0.05 * rng.standard_normal(mu.shape)).astype(np.float32)
+    _, lab, cnt = _kmeans_gpu(dev(X[None], torch.bfloat16), sv.SVGEAR_BF16, C, 0, dev(mu[None]))
+    nd = label_mismatches_are_ties(X, mu, lab[0])
+    assert nd <= 2, nd
+    np.testing.assert_array_equal(cnt[0], np.bincount(lab[0], minlength=C))
