@@ -9,12 +9,15 @@
 // error: rounding the centroid to bf16 moves x.mu by at most ||x|| ||mu - bf16(mu)||,
 // the fp32 accumulation by at most 2^-14 ||x|| ||bf16(mu)||, plus the
 // rounding of ||mu||^2 and of the epilogue FMA.  A single survivor is the exact
-// argmin; otherwise the survivors are re-decided with float64 distances
-// (smaller index on equal distance), so labels equal the exact argmin.
+// argmin; otherwise the token goes on a list that k_refine re-decides with
+// float64 distances (smaller index on equal distance), so labels equal the
+// exact argmin.
 //
 // Block of 12 warps: warp 0 allocates tensor memory and issues MMAs, warps 1-3
 // copy tiles (cp.async into the 128-byte-swizzled layout), warps 4-7 and 8-11
 // are two epilogue warpgroups that take alternate 256-column accumulator slots.
+// The epilogue reads each slot twice: a branch-free minimum pass, then a pass
+// that lists every column inside the window of the minimum.
 #include <algorithm>
 #include <cfloat>
 
@@ -32,6 +35,7 @@ constexpr int kThreads = 384;
 constexpr int kProducers = 96;
 constexpr int kCentBytesMax = 128 * 1024;
 constexpr int kSlotCols = 256;
+constexpr int kRefineInts = 4 + KC;   // h, row, n (-1 = overflow), pad, candidates
 
 __host__ __device__ inline int round16(int x) { return (x + 15) & ~15; }
 
@@ -104,44 +108,98 @@ __global__ void k_row_norms(const bf16* __restrict__ X, long long rows, float* _
   if (lane == 0) xn[r] = sqrtf(s) * 1.00001f;
 }
 
+// Per-token candidate state: minimum score, number of listed candidates and
+// an overflow flag in registers; the list (KC entries per epilogue thread,
+// strided by the 256 epilogue threads) in shared memory.
 struct Cands {
   float best;
-  int bc;
   int n;
   int over;
-  float s[KC];
-  int c[KC];
 };
 
-__device__ __forceinline__ void cand_init(Cands& st) {
-  st.best = INFINITY; st.bc = 0; st.n = 0; st.over = 0;
-}
-
-__device__ __forceinline__ void cand_compact(Cands& st, float W) {
+// Drop listed candidates that fell out of the window after `best` decreased.
+__device__ __forceinline__ void cand_compact(Cands& st, float W, float* ls, int* lc) {
   int m = 0;
-  for (int i = 0; i < st.n; ++i)
-    if (st.s[i] <= st.best + W) { st.s[m] = st.s[i]; st.c[m] = st.c[i]; ++m; }
+  for (int i = 0; i < min(st.n, KC); ++i) {
+    const float v = ls[i * 256];
+    if (v <= st.best + W) { ls[m * 256] = v; lc[m * 256] = lc[i * 256]; ++m; }
+  }
   st.n = m;
 }
 
-__device__ __forceinline__ void cand_add(Cands& st, float s, int c, float W) {
-  if (s < st.best || (s == st.best && c < st.bc)) { st.best = s; st.bc = c; }
-  if (st.n == KC) cand_compact(st, W);
-  if (st.n == KC) { st.over = 1; return; }
-  st.s[st.n] = s; st.c[st.n] = c; ++st.n;
+__device__ __forceinline__ void cand_push(Cands& st, float s, int c, float* ls, int* lc) {
+  if (st.n < KC) { ls[st.n * 256] = s; lc[st.n * 256] = c; }
+  else st.over = 1;
+  ++st.n;
 }
 
-template <int D>
-__device__ double exact_dist(const bf16* __restrict__ xrow, const float* __restrict__ mu) {
-  double acc = 0.0;
-#pragma unroll 4
-  for (int t = 0; t < D; t += 4) {
-    const float4 x = ld4(xrow + t);
-    const float4 m = *reinterpret_cast<const float4*>(mu + t);
-    double d0 = (double)x.x - m.x, d1 = (double)x.y - m.y, d2 = (double)x.z - m.z, d3 = (double)x.w - m.w;
-    acc = fma(d0, d0, acc); acc = fma(d1, d1, acc); acc = fma(d2, d2, acc); acc = fma(d3, d3, acc);
+// Pass 1: minimum score over 32 columns (branch-free).
+__device__ __forceinline__ float min32(const uint32_t (&v)[32], const float* cn) {
+  float m = INFINITY;
+#pragma unroll
+  for (int q = 0; q < 32; q += 4) {
+    const float4 n4 = *reinterpret_cast<const float4*>(cn + q);
+    const float a = fmaf(-2.f, __uint_as_float(v[q]), n4.x), b = fmaf(-2.f, __uint_as_float(v[q + 1]), n4.y);
+    const float c = fmaf(-2.f, __uint_as_float(v[q + 2]), n4.z), d = fmaf(-2.f, __uint_as_float(v[q + 3]), n4.w);
+    m = fminf(m, fminf(fminf(a, b), fminf(c, d)));
   }
-  return acc;
+  return m;
+}
+
+// Pass 2: list every column whose score is within the fixed threshold.
+template <int G>
+__device__ __forceinline__ void collect(Cands& st, const uint32_t (&v)[G], const float* cn, int cbase, int C,
+                                        float thr, float* ls, int* lc) {
+#pragma unroll
+  for (int q = 0; q < G; ++q) {
+    const float sq = fmaf(-2.f, __uint_as_float(v[q]), cn[q]);
+    if (sq <= thr && cbase + q < C) cand_push(st, sq, cbase + q, ls, lc);
+  }
+}
+
+// Rows the tensor-core pass left ambiguous: one warp per row computes float64
+// distances ||x - mu_c||^2 to each listed candidate (to every centroid when
+// the list overflowed) and keeps the smallest (smaller index on ties).
+template <int D>
+__global__ void __launch_bounds__(256) k_refine(const bf16* __restrict__ X, const float* __restrict__ cent,
+                                                int N, int C, const int* __restrict__ refine,
+                                                const int* __restrict__ count, int32_t* __restrict__ labels) {
+  constexpr int PER = D / 32;
+  const int lane = threadIdx.x & 31;
+  const int nw = gridDim.x * (blockDim.x >> 5);
+  const int total = *count;
+  for (int w = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); w < total; w += nw) {
+    const int* e = refine + (size_t)w * kRefineInts;
+    const int h = e[0], row = e[1], n = e[2];
+    float xv[PER];
+    {
+      const bf16* xr = X + ((size_t)h * N + row) * D + lane * PER;
+      if constexpr (PER == 4) {
+        const float4 v = ld4(xr);
+        xv[0] = v.x; xv[1] = v.y; xv[2] = v.z; xv[3] = v.w;
+      } else {
+        const float2 v = ld2(xr);
+        xv[0] = v.x; xv[1] = v.y;
+      }
+    }
+    const int cnt = n < 0 ? C : n;
+    double best = 1e300;
+    int bc = 0;
+    for (int i = 0; i < cnt; ++i) {
+      const int c = n < 0 ? i : e[3 + i];
+      const float* mu = cent + ((size_t)h * C + c) * D + lane * PER;
+      double acc = 0.0;
+#pragma unroll
+      for (int t = 0; t < PER; ++t) {
+        const double df = (double)xv[t] - (double)mu[t];
+        acc = fma(df, df, acc);
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+      if (acc < best || (acc == best && c < bc)) { best = acc; bc = c; }
+    }
+    if (lane == 0) labels[(size_t)h * N + row] = bc;
+  }
 }
 
 template <int D>
@@ -152,7 +210,8 @@ struct Smem {
   __host__ __device__ static int x_off(int Cpad) { return (Cpad * D * 2 + 1023) & ~1023; }
   __host__ __device__ static int cn_off(int Cpad) { return x_off(Cpad) + 2 * kXBytes; }
   __host__ __device__ static int merge_off(int Cpad) { return cn_off(Cpad) + ((Cpad * 4 + 15) & ~15); }
-  __host__ __device__ static int bar_off(int Cpad) { return merge_off(Cpad) + BM * (4 + 2 * KC) * 4; }
+  __host__ __device__ static int list_off(int Cpad) { return merge_off(Cpad) + BM * 4 * 4; }
+  __host__ __device__ static int bar_off(int Cpad) { return list_off(Cpad) + 2 * KC * 256 * 4; }
   // at least 120 KB so that only one block (and one 512-column tensor-memory
   // allocation) lives on an SM
   static int total(int Cpad) { return std::max(bar_off(Cpad) + 16 * 8 + 1024, 120 * 1024); }
@@ -163,7 +222,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     k_assign_tc(const bf16* __restrict__ X, const bf16* __restrict__ cb, const float* __restrict__ cnorm,
                 const Bounds* __restrict__ bounds, const float* __restrict__ xnorm,
                 const float* __restrict__ cent, int N, int C, int Cpad, int tiles_per_cta,
-                int32_t* __restrict__ labels, int* status) {
+                int32_t* __restrict__ labels, int* __restrict__ refine, int* __restrict__ refine_count,
+                int* status) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   using S = Smem<D>;
@@ -171,6 +231,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* x_s = smem + S::x_off(Cpad);
   float* cn_s = reinterpret_cast<float*>(smem + S::cn_off(Cpad));
   int* merge = reinterpret_cast<int*>(smem + S::merge_off(Cpad));
+  float* list_s = reinterpret_cast<float*>(smem + S::list_off(Cpad));
+  int* list_c = reinterpret_cast<int*>(smem + S::list_off(Cpad) + KC * 256 * 4);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + S::bar_off(Cpad));
   uint64_t* cent_full = bars + 0;
   uint64_t* x_full = bars + 1;     // [2]
@@ -276,16 +338,16 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int wg = (warp - 4) >> 2;           // 0 or 1
     const int r = ((warp & 3) << 5) + lane;   // TMEM lane == tile row
     const Bounds bd = bounds[h];
-    const float* ch = cent + (size_t)h * C * D;
-    const bf16* Xh = X + (size_t)h * N * D;
     for (int t = 0; t < nt; ++t) {
       const int row = (t0 + t) * BM + r;
       const float xn = row < N ? xnorm[(size_t)h * N + row] : 0.f;
       const float B = 2.f * xn * (bd.dmax + 6.1035e-5f * bd.mmax) +
                       9.5367e-7f * (bd.nmax + 2.f * xn * bd.mmax) + 1e-30f;
       const float W = 2.f * B;
-      Cands st;
-      cand_init(st);
+      const int et = threadIdx.x - 128;  // epilogue thread 0..255
+      float* ls = list_s + et;
+      int* lc = list_c + et;
+      Cands st{INFINITY, 0, 0};
       bool mine = false;
       for (int j = 0; j < nchunk; ++j) {
         const int g = t * nchunk + j, slot = g & 1, use = g >> 1;
@@ -295,75 +357,86 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc::tc_fence_after();
         const int n0 = j * kSlotCols, nj = min(kSlotCols, Cpad - n0);
         const uint32_t base = tc::taddr(tmem, (uint32_t)((warp & 3) << 5), (uint32_t)(slot * kSlotCols));
-        int c0 = 0;
-        for (; c0 + 32 <= nj; c0 += 32) {
+        const int n32 = nj & ~31;
+        // pass 1: chunk minimum (padding columns score +inf)
+        float m = INFINITY;
+        for (int c0 = 0; c0 < n32; c0 += 32) {
           uint32_t v[32];
           tc::tmem_ld32(base + (uint32_t)c0, v);
           tc::tmem_ld_wait();
-#pragma unroll
-          for (int q = 0; q < 32; ++q) {
-            const int c = n0 + c0 + q;
-            const float s = fmaf(-2.f, __uint_as_float(v[q]), cn_s[c]);
-            if (c < C && s <= st.best + W) cand_add(st, s, c, W);
-          }
+          m = fminf(m, min32(v, cn_s + n0 + c0));
         }
-        if (c0 < nj) {  // 16-column tail
+        if (n32 < nj) {
           uint32_t v[16];
-          tc::tmem_ld16(base + (uint32_t)c0, v);
+          tc::tmem_ld16(base + (uint32_t)n32, v);
           tc::tmem_ld_wait();
 #pragma unroll
-          for (int q = 0; q < 16; ++q) {
-            const int c = n0 + c0 + q;
-            const float s = fmaf(-2.f, __uint_as_float(v[q]), cn_s[c]);
-            if (c < C && s <= st.best + W) cand_add(st, s, c, W);
-          }
+          for (int q = 0; q < 16; ++q) m = fminf(m, fmaf(-2.f, __uint_as_float(v[q]), cn_s[n0 + n32 + q]));
+        }
+        if (m < st.best) {
+          st.best = m;
+          if (st.n) cand_compact(st, W, ls, lc);
+        }
+        // pass 2: every column within the window of the running minimum
+        const float thr = st.best + W;
+        for (int c0 = 0; c0 < n32; c0 += 32) {
+          uint32_t v[32];
+          tc::tmem_ld32(base + (uint32_t)c0, v);
+          tc::tmem_ld_wait();
+          collect<32>(st, v, cn_s + n0 + c0, n0 + c0, C, thr, ls, lc);
+        }
+        if (n32 < nj) {
+          uint32_t v[16];
+          tc::tmem_ld16(base + (uint32_t)n32, v);
+          tc::tmem_ld_wait();
+          collect<16>(st, v, cn_s + n0 + n32, n0 + n32, C, thr, ls, lc);
         }
         tc::tc_fence_before();
         tc::mbar_arrive(acc_empty + slot);
       }
       // on abort keep walking the tiles (waits now return at once) so that
       // both warpgroups pass the same named barriers
-      // combine the two warpgroups' partial results when both saw this tile
       bool finalize = mine;
       if (nchunk >= 2) {
-        int* mrow = merge + r * (4 + 2 * KC);
-        if (wg == 1) {
-          mrow[0] = __float_as_int(st.best); mrow[1] = st.bc; mrow[2] = st.n; mrow[3] = st.over;
-          for (int i = 0; i < st.n; ++i) { mrow[4 + i] = __float_as_int(st.s[i]); mrow[4 + KC + i] = st.c[i]; }
-        }
+        int* mrow = merge + r * 4;
+        if (wg == 1) { mrow[0] = __float_as_int(st.best); mrow[2] = st.n; mrow[3] = st.over; }
         asm volatile("bar.sync 1, 256;" ::: "memory");
         if (wg == 0) {
           const float ob = __int_as_float(mrow[0]);
-          const int obc = mrow[1], on = mrow[2];
+          const int on = mrow[2];
           st.over |= mrow[3];
-          if (ob < st.best || (ob == st.best && obc < st.bc)) { st.best = ob; st.bc = obc; }
-          for (int i = 0; i < on; ++i) cand_add(st, __int_as_float(mrow[4 + i]), mrow[4 + KC + i], W);
+          if (ob < st.best) {
+            st.best = ob;
+            if (st.n) cand_compact(st, W, ls, lc);
+          }
+          const float thr = st.best + W;
+          for (int i = 0; i < min(on, KC); ++i) {
+            const float os = list_s[i * 256 + et + 128];
+            if (os <= thr) cand_push(st, os, list_c[i * 256 + et + 128], ls, lc);
+          }
+          if (on > KC) st.over = 1;
         }
         asm volatile("bar.sync 1, 256;" ::: "memory");
         finalize = wg == 0;
       }
       if (!finalize || row >= N || *abort_flag) continue;
-      cand_compact(st, W);
-      int label = st.bc;
-      if (st.over || st.n > 1) {
-        const bf16* xr = Xh + (size_t)row * D;
-        double bestd = 1e300;
-        int bestc = 0;
-        if (st.over) {
-          for (int c = 0; c < C; ++c) {
-            const double dd = exact_dist<D>(xr, ch + (size_t)c * D);
-            if (dd < bestd) { bestd = dd; bestc = c; }
-          }
-        } else {
-          for (int i = 0; i < st.n; ++i) {
-            const int c = st.c[i];
-            const double dd = exact_dist<D>(xr, ch + (size_t)c * D);
-            if (dd < bestd || (dd == bestd && c < bestc)) { bestd = dd; bestc = c; }
-          }
-        }
-        label = bestc;
+      // the listed candidate with the smallest score (smaller index on ties)
+      cand_compact(st, W, ls, lc);
+      int label = 0;
+      float bs = INFINITY;
+      for (int i = 0; i < min(st.n, KC); ++i) {
+        const float v = ls[i * 256];
+        const int c = lc[i * 256];
+        if (v < bs || (v == bs && c < label)) { bs = v; label = c; }
       }
       labels[(size_t)h * N + row] = label;
+      if (st.n > 1 || st.over) {
+        // several centroids within the bound: decided later in float64
+        const int k = atomicAdd(refine_count, 1);
+        int* e = refine + (size_t)k * kRefineInts;
+        e[0] = h; e[1] = row; e[2] = st.over ? -1 : st.n;
+        for (int i = 0; i < min(st.n, KC); ++i) e[3 + i] = lc[i * 256];
+      }
     }
   }
 
@@ -384,22 +457,34 @@ bool kmeans_tc_supported(int d, int C) {
 }
 
 // Workspace: token norms [H,N] first (they only depend on H, N), then the
-// per-iteration centroid copy, norms and bounds.
-static size_t tc_layout(int H, int N, int d, int C, bf16** cb, float** cn, Bounds** bd, float** xn,
-                        void* ws) {
+// per-iteration centroid copy, norms and bounds, and the list of rows left
+// for the float64 pass with its counter.
+struct TcWs {
+  float* xn;
+  bf16* cb;
+  float* cn;
+  Bounds* bd;
+  int* refine;
+  int* refine_count;
+};
+
+static size_t tc_layout(int H, int N, int d, int C, TcWs* out, void* ws) {
   Carve cv(ws);
   const int Cpad = round16(C);
-  float* e = cv.take<float>((size_t)H * N);
-  bf16* a = cv.take<bf16>((size_t)H * Cpad * d);
-  float* b = cv.take<float>((size_t)H * Cpad);
-  Bounds* c = cv.take<Bounds>(H);
-  if (cb) { *cb = a; *cn = b; *bd = c; *xn = e; }
+  TcWs w;
+  w.xn = cv.take<float>((size_t)H * N);
+  w.cb = cv.take<bf16>((size_t)H * Cpad * d);
+  w.cn = cv.take<float>((size_t)H * Cpad);
+  w.bd = cv.take<Bounds>(H);
+  w.refine = cv.take<int>((size_t)H * N * kRefineInts);
+  w.refine_count = cv.take<int>(1);
+  if (out) *out = w;
   return cv.used();
 }
 
 size_t kmeans_tc_ws_bytes(int H, int N, int d, int C) {
   if (!kmeans_tc_supported(d, C)) return 0;
-  return tc_layout(H, N, d, C, nullptr, nullptr, nullptr, nullptr, nullptr);
+  return tc_layout(H, N, d, C, nullptr, nullptr);
 }
 
 cudaError_t kmeans_tc_prepare_rows(const void* Xv, int H, int N, int d, void* ws, cudaStream_t st) {
@@ -413,28 +498,33 @@ cudaError_t kmeans_tc_prepare_rows(const void* Xv, int H, int N, int d, void* ws
 
 cudaError_t kmeans_assign_tc(const void* Xv, int H, int N, int d, int C, const float* cent,
                              int32_t* labels, void* ws, cudaStream_t st) {
-  bf16 *cb; float *cn, *xn; Bounds* bd;
-  tc_layout(H, N, d, C, &cb, &cn, &bd, &xn, ws);
+  TcWs w;
+  tc_layout(H, N, d, C, &w, ws);
   const int Cpad = round16(C);
   const bf16* X = static_cast<const bf16*>(Xv);
   const int T = (N + BM - 1) / BM;
-  int tpc = std::max(1, std::min(16, (int)((long long)H * T / (2 * 148))));
+  const int tpc = std::max(1, std::min(16, (int)((long long)H * T / (2 * 148))));
   const int gx = (T + tpc - 1) / tpc;
-  cudaError_t e;
+  cudaError_t e = cudaMemsetAsync(w.refine_count, 0, sizeof(int), st);
+  if (e != cudaSuccess) return e;
   if (d == 128) {
-    k_prep_centroids<128><<<H, 256, 0, st>>>(cent, C, Cpad, cb, cn, bd); note_launch();
+    k_prep_centroids<128><<<H, 256, 0, st>>>(cent, C, Cpad, w.cb, w.cn, w.bd); note_launch();
     const int smem = Smem<128>::total(Cpad);
     e = cudaFuncSetAttribute(k_assign_tc<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
-    k_assign_tc<128><<<dim3(gx, H), kThreads, smem, st>>>(X, cb, cn, bd, xn, cent, N, C, Cpad, tpc, labels,
-                                                           status_word()); note_launch();
+    k_assign_tc<128><<<dim3(gx, H), kThreads, smem, st>>>(X, w.cb, w.cn, w.bd, w.xn, cent, N, C, Cpad, tpc,
+                                                           labels, w.refine, w.refine_count, status_word());
+    note_launch();
+    k_refine<128><<<148 * 8, 256, 0, st>>>(X, cent, N, C, w.refine, w.refine_count, labels); note_launch();
   } else {
-    k_prep_centroids<64><<<H, 256, 0, st>>>(cent, C, Cpad, cb, cn, bd); note_launch();
+    k_prep_centroids<64><<<H, 256, 0, st>>>(cent, C, Cpad, w.cb, w.cn, w.bd); note_launch();
     const int smem = Smem<64>::total(Cpad);
     e = cudaFuncSetAttribute(k_assign_tc<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
-    k_assign_tc<64><<<dim3(gx, H), kThreads, smem, st>>>(X, cb, cn, bd, xn, cent, N, C, Cpad, tpc, labels,
-                                                          status_word()); note_launch();
+    k_assign_tc<64><<<dim3(gx, H), kThreads, smem, st>>>(X, w.cb, w.cn, w.bd, w.xn, cent, N, C, Cpad, tpc,
+                                                          labels, w.refine, w.refine_count, status_word());
+    note_launch();
+    k_refine<64><<<148 * 8, 256, 0, st>>>(X, cent, N, C, w.refine, w.refine_count, labels); note_launch();
   }
   return cudaGetLastError();
 }
