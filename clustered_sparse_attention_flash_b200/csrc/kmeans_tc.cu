@@ -353,7 +353,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int g = t * nchunk + j, slot = g & 1, use = g >> 1;
         if (slot != wg) continue;
         mine = true;
-        if (!tc::mbar_wait(acc_full + slot, use & 1, abort_flag, status)) break;
+        if (!tc::mbar_wait_warp(acc_full + slot, use & 1, abort_flag, status)) break;
         tc::tc_fence_after();
         const int n0 = j * kSlotCols, nj = min(kSlotCols, Cpad - n0);
         const uint32_t base = tc::taddr(tmem, (uint32_t)((warp & 3) << 5), (uint32_t)(slot * kSlotCols));
@@ -444,7 +444,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   if (warp == 0) {
     tc::tc_fence_after();
-    tc::mbar_wait(done, 0, abort_flag, status);
+    tc::mbar_wait_warp(done, 0, abort_flag, status);
+    __syncwarp();
     tc::tmem_dealloc(tmem, 512);
   }
 }
