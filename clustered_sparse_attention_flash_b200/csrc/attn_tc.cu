@@ -390,14 +390,24 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t va = tc::smem_u32(smem + S::v_off + st * S::kKTile);
       const bf16* ksrc = exact ? Kh : (p == 0 ? kb_hi : kb_lo) + cbase;
       const bf16* vsrc = exact ? Vh : (p == 0 ? vb_hi : vb_lo) + cbase;
-      for (int e = lane; e < BN * CPR; e += 32) {
-        const int r = e / CPR, c = e % CPR;
-        const int row = idx[r];
-        const uint32_t nb = row >= 0 ? 16u : 0u;
-        const size_t off = (size_t)(row >= 0 ? row : 0) * D + c * 8;
-        const uint32_t so = tc::sw128_offset(r, c, BN);
-        tc::cp_async16(ka + so, ksrc + off, nb);
-        tc::cp_async16(va + so, vsrc + off, nb);
+      {
+        // lane -> (row offset, 16-byte chunk); each warp instruction copies
+        // RPI whole rows (coalesced); row indices are read up front so the
+        // copies issue back to back
+        constexpr int RPI = 32 / CPR, NIT = BN / RPI;
+        const int rofs = lane / CPR, c = lane % CPR;
+        int rows[NIT];
+#pragma unroll
+        for (int i = 0; i < NIT; ++i) rows[i] = idx[i * RPI + rofs];
+#pragma unroll
+        for (int i = 0; i < NIT; ++i) {
+          const int row = rows[i];
+          const uint32_t nb = row >= 0 ? 16u : 0u;
+          const size_t off = (size_t)(row >= 0 ? row : 0) * D + c * 8;
+          const uint32_t so = tc::sw128_offset(i * RPI + rofs, c, BN);
+          tc::cp_async16(ka + so, ksrc + off, nb);
+          tc::cp_async16(va + so, vsrc + off, nb);
+        }
       }
       tc::cp_async_wait_all();
       tc::fence_proxy_async();
@@ -417,13 +427,16 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!tc::mbar_wait_warp(s_full + x * 2 + b, (j >> 1) & 1, abort_flag, status)) { ok = false; break; }
       tc::tc_fence_after();
       float xs[BN];
-#pragma unroll
-      for (int q = 0; q < BN / 32; ++q) {
-        uint32_t v[32];
-        tc::tmem_ld32(tmem + lane_base + scol + (uint32_t)(b * 64 + q * 32), v);
+      {
+        uint32_t v0[32], v1[32];
+        tc::tmem_ld32(tmem + lane_base + scol + (uint32_t)(b * 64), v0);
+        tc::tmem_ld32(tmem + lane_base + scol + (uint32_t)(b * 64 + 32), v1);
         tc::tmem_ld_wait();
 #pragma unroll
-        for (int i = 0; i < 32; ++i) xs[q * 32 + i] = __uint_as_float(v[i]) * scale2;
+        for (int i = 0; i < 32; ++i) {
+          xs[i] = __uint_as_float(v0[i]) * scale2;
+          xs[32 + i] = __uint_as_float(v1[i]) * scale2;
+        }
       }
       // bias / mask of this stage: acquire the producers' writes through the
       // stage's full barrier (its next phase needs this tile's P first)
@@ -436,9 +449,15 @@ __global__ void __launch_bounds__(kThreads, 1)
           xs[i] += b4.x; xs[i + 1] += b4.y; xs[i + 2] += b4.z; xs[i + 3] += b4.w;
         }
       }
-      float mx = -INFINITY;
+      float mx;
+      {  // 8 independent chains instead of one 64-long chain
+        float m8[8];
 #pragma unroll
-      for (int i = 0; i < BN; ++i) mx = fmaxf(mx, xs[i]);
+        for (int k = 0; k < 8; ++k) m8[k] = xs[k];
+#pragma unroll
+        for (int i = 8; i < BN; ++i) m8[i & 7] = fmaxf(m8[i & 7], xs[i]);
+        mx = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])), fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
+      }
       // lazy rescale: a row whose maximum grew by more than 2^8 rescales O and
       // l.  The tensor-memory accesses are warp-collective, so the warp
       // rescales together (factor 1 for rows that do not need it).
@@ -463,21 +482,21 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       if (grow) m_used = mx;
       const float mref = m_used == -INFINITY ? 0.f : m_used;
-      float rs = 0.f;
+      float r8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
 #pragma unroll
       for (int q = 0; q < BN / 32; ++q) {
         uint32_t pk[16];
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
           const float p0 = ex2(xs[q * 32 + 2 * i] - mref), p1 = ex2(xs[q * 32 + 2 * i + 1] - mref);
-          rs += p0 + p1;
+          r8[i & 7] += p0 + p1;
           pk[i] = pack_bf16(p0, p1);
         }
         // P over the first 32 columns of this S buffer (already read above)
         tc::tmem_st16(tmem + lane_base + scol + (uint32_t)(b * 64 + q * 16), pk);
       }
       tc::tmem_st_wait();
-      l += rs;
+      l += ((r8[0] + r8[1]) + (r8[2] + r8[3])) + ((r8[4] + r8[5]) + (r8[6] + r8[7]));
       tc::tc_fence_before();
       tc::mbar_arrive(p_full + x * 2 + b);
     }
