@@ -100,7 +100,7 @@ FwdLayout layout(const svgear_params* p, void* ws) {
   size_t sb = kmeans_ws_bytes(H, Nq, d, Cq);
   sb = std::max(sb, kmeans_ws_bytes(H, Nk, d, Ck));
   sb = std::max(sb, block_error_ws_bytes(H, Cq, Ck));
-  sb = std::max(sb, attn_ws_bytes(H, Nq, d, Cq, Ck));
+  sb = std::max(sb, attn_ws_bytes(H, Nq, Nk, d, Cq, Ck));
   L.scratch = cv.take<char>(sb);
   L.scratch_bytes = sb;
   L.total = cv.used();
@@ -213,7 +213,7 @@ int svgear_route(const float* E, const int32_t* k_counts, const int32_t* q_count
 
 size_t svgear_hybrid_attn_workspace_size(const svgear_params* p) {
   if (check_params(p)) return 0;
-  return attn_ws_bytes(p->H, p->Nq, p->d, p->Cq, p->Ck);
+  return attn_ws_bytes(p->H, p->Nq, p->Nk, p->d, p->Cq, p->Ck);
 }
 
 int svgear_hybrid_attn(const void* Qp, const void* Kp, const void* Vp, const int32_t* q_off,
@@ -227,7 +227,7 @@ int svgear_hybrid_attn(const void* Qp, const void* Kp, const void* Vp, const int
   if (!aligned16(Qp) || !aligned16(Kp) || !aligned16(Vp) || !aligned16(O) || !aligned16(Kbar) ||
       !aligned16(Vbar))
     return SVGEAR_ERR_INVALID;
-  if (!ws || ws_bytes < attn_ws_bytes(p->H, p->Nq, p->d, p->Cq, p->Ck)) return SVGEAR_ERR_WORKSPACE;
+  if (!ws || ws_bytes < attn_ws_bytes(p->H, p->Nq, p->Nk, p->d, p->Cq, p->Ck)) return SVGEAR_ERR_WORKSPACE;
   return cuda_status(attn_run(Qp, Kp, Vp, q_off, k_off, perm_q, Kbar, Vbar, sel, n_sel, p->dtype,
                               p->H, p->Nq, p->Nk, p->d, p->Cq, p->Ck, eff_scale(p), O, ws, S(stream)));
 }

@@ -180,12 +180,12 @@ void launch_simt(const void* Qp, const void* Kp, const void* Vp, const int32_t* 
 
 }  // namespace
 
-size_t attn_ws_bytes(int H, int Nq, int d, int Cq, int Ck) {
+size_t attn_ws_bytes(int H, int Nq, int Nk, int d, int Cq, int Ck) {
   Carve cv(nullptr);
   const int tmax = (Nq + kBQ - 1) / kBQ + Cq;
   cv.take<int2>((size_t)H * tmax);
   cv.take<int32_t>(H);
-  cv.take<char>(attn_tc_ws_bytes(H, Nq, d, Cq, Ck));
+  cv.take<char>(attn_tc_ws_bytes(H, Nq, Nk, d, Cq, Ck));
   return cv.used();
 }
 
@@ -198,7 +198,7 @@ cudaError_t attn_run(const void* Qp, const void* Kp, const void* Vp, const int32
   const int tmax = (Nq + kBQ - 1) / kBQ + Cq;
   int2* tiles = cv.take<int2>((size_t)H * tmax);
   int32_t* ntiles = cv.take<int32_t>(H);
-  void* tcws = cv.take<char>(attn_tc_ws_bytes(H, Nq, d, Cq, Ck));
+  void* tcws = cv.take<char>(attn_tc_ws_bytes(H, Nq, Nk, d, Cq, Ck));
   if (dtype == DT_BF16 && attn_tc_supported(d, Ck))
     return attn_tc_run(Qp, Kp, Vp, q_off, k_off, perm_q, Kbar, Vbar, sel, n_sel, H, Nq, Nk, d, Cq,
                        Ck, scale, O, tcws, st);

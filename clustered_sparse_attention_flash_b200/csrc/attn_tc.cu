@@ -16,15 +16,21 @@
 //     float32 centroids enter as bf16 hi + lo pairs (two MMAs each for S and
 //     for P.V), so their rounding stays near 2^-17 instead of 2^-9; such a
 //     tile occupies two ring stages (hi, then lo).
-// Key tiles flow through a four-stage ring of 64-row K and V tiles.
+// Key tiles flow through a four-stage ring of 64-row K and V tiles.  Keys and
+// values are staged in an "8-row group" layout (each key cluster padded to a
+// multiple of 8 rows, each group of 8 rows stored as [16-byte chunk][row]),
+// which is directly a no-swizzle UMMA operand (K-major for K, MN-major for
+// V); a stage is therefore one or a few contiguous runs, each moved by a
+// single cp.async.bulk completing on the stage's mbarrier.  Padding rows are
+// masked through the stage's bias vector.
 // Warp roles (12 warps):
 //   warp 0      tensor-memory allocation, MMA issue (one thread): per key
 //               tile S_A, S_B = Q_{A,B} K^T into double-buffered S, then
 //               O_{A,B} += P V of the previous tile with P read from tensor
 //               memory;
-//   warps 1-3   producers: cp.async gathers of Q, K, V rows into the
-//               128-byte-swizzled layout, up to three stages in flight,
-//               bias vectors; named barriers 2 and 3 order them;
+//   warps 1-3   load the two query tiles (cp.async into the 128-byte-swizzled
+//               layout), then produce every third key stage each (bulk copies
+//               issued by one lane, bias vectors by the whole warp);
 //   warps 4-7   softmax of tile A, warps 8-11 softmax of tile B (thread =
 //               query row): row max, lazy rescale of O when the max grows by
 //               more than 2^8, P = 2^(x - m) in bf16 written over the S
@@ -52,7 +58,7 @@ constexpr int kStages = 4;
 constexpr int kUnitRows = 2 * BQ;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr uint32_t kColS = 0, kColO = 256;
-constexpr int kMaxRanges = 2048;  // routed clusters staged in shared memory
+constexpr int kMaxRanges = 1024;  // routed clusters staged in shared memory
 
 __device__ __forceinline__ float ex2(float x) {
   float y;
@@ -66,29 +72,97 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   return r;
 }
 
-// bf16 hi/lo copies of the key / value centroids (x = hi + lo + O(2^-17 x);
-// rows padded to a multiple of 64 with zeros) and log2 of the cluster sizes
-// (-inf for empty or padding).
+// Byte offset of (row, 16-byte chunk) in the 8-row group layout.
+template <int D>
+__host__ __device__ __forceinline__ size_t g8_offset(size_t row, int chunk) {
+  return (row >> 3) * (size_t)(8 * D * 2) + (size_t)chunk * 128u + (row & 7) * 16u;
+}
+
+// bf16 hi/lo copies of the key / value centroids (x = hi + lo + O(2^-17 x)),
+// in the 8-row group layout with rows padded to a multiple of 64 (zeros),
+// and log2 of the cluster sizes (-inf for empty or padding).
 template <int D>
 __global__ void k_prep_comp(const float* __restrict__ Kbar, const float* __restrict__ Vbar,
-                            const int32_t* __restrict__ k_off, int Ck, int Ckpad, bf16* __restrict__ kh,
-                            bf16* __restrict__ kl, bf16* __restrict__ vh, bf16* __restrict__ vl,
+                            const int32_t* __restrict__ k_off, int Ck, int Ckpad, uint8_t* __restrict__ kh,
+                            uint8_t* __restrict__ kl, uint8_t* __restrict__ vh, uint8_t* __restrict__ vl,
                             float* __restrict__ lc2) {
   const int h = blockIdx.y, c = blockIdx.x;
   const bool ok = c < Ck;
+  const size_t hb = (size_t)h * Ckpad * D * 2;
   for (int t = threadIdx.x; t < D; t += blockDim.x) {
-    const size_t src = ((size_t)h * Ck + c) * D + t, dst = ((size_t)h * Ckpad + c) * D + t;
+    const size_t src = ((size_t)h * Ck + c) * D + t;
+    const size_t dst = hb + g8_offset<D>(c, t >> 3) + (t & 7) * 2;
     const float k = ok ? Kbar[src] : 0.f, v = ok ? Vbar[src] : 0.f;
     const bf16 k1 = __float2bfloat16_rn(k), v1 = __float2bfloat16_rn(v);
-    kh[dst] = k1;
-    kl[dst] = __float2bfloat16_rn(k - __bfloat162float(k1));
-    vh[dst] = v1;
-    vl[dst] = __float2bfloat16_rn(v - __bfloat162float(v1));
+    *reinterpret_cast<bf16*>(kh + dst) = k1;
+    *reinterpret_cast<bf16*>(kl + dst) = __float2bfloat16_rn(k - __bfloat162float(k1));
+    *reinterpret_cast<bf16*>(vh + dst) = v1;
+    *reinterpret_cast<bf16*>(vl + dst) = __float2bfloat16_rn(v - __bfloat162float(v1));
   }
   if (threadIdx.x == 0) {
     int n = 0;
     if (ok) n = k_off[(size_t)h * (Ck + 1) + c + 1] - k_off[(size_t)h * (Ck + 1) + c];
     lc2[(size_t)h * Ckpad + c] = n > 0 ? log2f((float)n) : -INFINITY;
+  }
+}
+
+// poff[h][c]: first padded row of key cluster c (sizes rounded up to 8).
+__global__ void k_pad_offsets(const int32_t* __restrict__ k_off, int Ck, int32_t* __restrict__ poff) {
+  __shared__ int32_t wtot[32];
+  __shared__ int32_t carry;
+  const int h = blockIdx.x, lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+  const int32_t* off = k_off + (size_t)h * (Ck + 1);
+  int32_t* po = poff + (size_t)h * (Ck + 1);
+  if (threadIdx.x == 0) carry = 0;
+  __syncthreads();
+  for (int c0 = 0; c0 < Ck; c0 += blockDim.x) {
+    const int c = c0 + threadIdx.x;
+    const int n = c < Ck ? ((off[c + 1] - off[c] + 7) & ~7) : 0;
+    int v = n;
+    for (int o = 1; o < 32; o <<= 1) {
+      const int u = __shfl_up_sync(0xffffffffu, v, o);
+      if (lane >= o) v += u;
+    }
+    if (lane == 31) wtot[w] = v;
+    __syncthreads();
+    if (w == 0) {
+      int t = (lane < (int)(blockDim.x >> 5)) ? wtot[lane] : 0;
+      for (int o = 1; o < 32; o <<= 1) {
+        const int u = __shfl_up_sync(0xffffffffu, t, o);
+        if (lane >= o) t += u;
+      }
+      wtot[lane] = t;
+    }
+    __syncthreads();
+    if (c < Ck) po[c] = carry + v - n + (w > 0 ? wtot[w - 1] : 0);
+    __syncthreads();
+    if (threadIdx.x == 0) carry += wtot[(blockDim.x >> 5) - 1];
+    __syncthreads();
+  }
+  if (threadIdx.x == 0) po[Ck] = carry;
+}
+
+// Key / value rows of cluster c (row-major, cluster order) into the padded
+// 8-row group layout; padding rows are zero.
+template <int D>
+__global__ void k_pack(const bf16* __restrict__ Kp, const bf16* __restrict__ Vp, const int32_t* __restrict__ k_off,
+                       const int32_t* __restrict__ poff, int Nk, int Ck, size_t npad, uint8_t* __restrict__ kpk,
+                       uint8_t* __restrict__ vpk) {
+  constexpr int CPR = D / 8;
+  const int h = blockIdx.y, c = blockIdx.x;
+  const int beg = k_off[(size_t)h * (Ck + 1) + c], len = k_off[(size_t)h * (Ck + 1) + c + 1] - beg;
+  const int pbeg = poff[(size_t)h * (Ck + 1) + c], plen = (len + 7) & ~7;
+  const size_t hb = (size_t)h * npad * D * 2;
+  const uint4* ks = reinterpret_cast<const uint4*>(Kp + ((size_t)h * Nk + beg) * D);
+  const uint4* vs = reinterpret_cast<const uint4*>(Vp + ((size_t)h * Nk + beg) * D);
+  for (int e = threadIdx.x; e < plen * CPR; e += blockDim.x) {
+    const int r = e / CPR, ch = e % CPR;
+    const uint4 z = make_uint4(0, 0, 0, 0);
+    const uint4 kv = r < len ? ks[(size_t)r * CPR + ch] : z;
+    const uint4 vv = r < len ? vs[(size_t)r * CPR + ch] : z;
+    const size_t o = hb + g8_offset<D>((size_t)(pbeg + r), ch);
+    *reinterpret_cast<uint4*>(kpk + o) = kv;
+    *reinterpret_cast<uint4*>(vpk + o) = vv;
   }
 }
 
@@ -142,37 +216,40 @@ struct AttnSmem {
   static constexpr int q_off = 0;             // [2] query tiles
   static constexpr int k_off = q_off + 2 * kQTile;
   static constexpr int v_off = k_off + kStages * kKTile;
-  static constexpr int idx_off = v_off + kStages * kKTile;
-  static constexpr int bias_off = idx_off + kStages * BN * 4;
+  static constexpr int bias_off = v_off + kStages * kKTile;
   static constexpr int flag_off = bias_off + kStages * BN * 4;
   static constexpr int bits_off = flag_off + 64;
-  static constexpr int rng_off = bits_off + kMaxCkBits / 8;   // [2][kMaxRanges] start, prefix
-  static constexpr int bar_off = rng_off + 2 * kMaxRanges * 4 + 16;
+  static constexpr int rng_off = bits_off + kMaxCkBits / 8;   // [3][kMaxRanges] start, prefix, len
+  static constexpr int pc_off = rng_off + 3 * kMaxRanges * 4 + 16;  // [producer warp][8] piece lists
+  static constexpr int bar_off = pc_off + 3 * 8 * 4 * 4;
   static constexpr int total = bar_off + 40 * 8 + 1024;
 };
 
 template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
-    k_attn_tc(const bf16* __restrict__ Qp, const bf16* __restrict__ Kp, const bf16* __restrict__ Vp,
-              const int32_t* __restrict__ q_off, const int32_t* __restrict__ k_off,
-              const int32_t* __restrict__ perm_q, const bf16* __restrict__ kb_hi,
-              const bf16* __restrict__ kb_lo, const bf16* __restrict__ vb_hi, const bf16* __restrict__ vb_lo,
+    k_attn_tc(const bf16* __restrict__ Qp, const uint8_t* __restrict__ kpk, const uint8_t* __restrict__ vpk,
+              size_t npad, const int32_t* __restrict__ q_off, const int32_t* __restrict__ k_off,
+              const int32_t* __restrict__ poff, const int32_t* __restrict__ perm_q,
+              const uint8_t* __restrict__ kb_hi, const uint8_t* __restrict__ kb_lo,
+              const uint8_t* __restrict__ vb_hi, const uint8_t* __restrict__ vb_lo,
               const float* __restrict__ lc2, const int32_t* __restrict__ sel,
               const int32_t* __restrict__ n_sel, const int2* __restrict__ tiles,
               const int32_t* __restrict__ ntiles, int tmax, int Nq, int Nk, int Cq, int Ck, int Ckpad,
               float scale2, bf16* __restrict__ O, int* status) {
   using S = AttnSmem<D>;
   constexpr int CPR = D / 8;  // 16-byte chunks per row
+  constexpr uint32_t kGroup = 8 * D * 2;  // bytes of one 8-row group
   const int h = blockIdx.y;
   if ((int)blockIdx.x >= ntiles[h]) return;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  int* idx_s = reinterpret_cast<int*>(smem + S::idx_off);         // [stage][BN] source rows
   float* bias_s = reinterpret_cast<float*>(smem + S::bias_off);   // [stage][BN] log2 biases
   int* flag_s = reinterpret_cast<int*>(smem + S::flag_off);       // [stage]: 1 = apply bias
   uint32_t* bits = reinterpret_cast<uint32_t*>(smem + S::bits_off);
-  int* rng_start = reinterpret_cast<int*>(smem + S::rng_off);  // first key row of routed range i
-  int* rng_cum = rng_start + kMaxRanges;                        // keys in ranges [0, i)
+  int* rng_start = reinterpret_cast<int*>(smem + S::rng_off);  // first padded row of routed range i
+  int* rng_cum = rng_start + kMaxRanges;                        // padded rows in ranges [0, i)
+  int* rng_len = rng_cum + kMaxRanges + 4;                      // keys in range i
+  int4* pieces = reinterpret_cast<int4*>(smem + S::pc_off);     // stage row group, global row, groups, valid
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + S::bar_off);
   uint64_t* q_full = bars + 0;
   uint64_t* kv_full = bars + 1;    // [kStages]
@@ -199,7 +276,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (threadIdx.x == 0) {
     tc::mbar_init(q_full, kProducers);
     for (int i = 0; i < kStages; ++i) {
-      tc::mbar_init(kv_full + i, 32);  // one producer warp fills a stage
+      tc::mbar_init(kv_full + i, 1);  // one arrival carrying the stage's byte count
       tc::mbar_init(kv_empty + i, 1);
     }
     for (int i = 0; i < 4; ++i) {
@@ -213,12 +290,13 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
   __syncthreads();
   long long lex_part = 0;
+  const int32_t* pof = poff + (size_t)h * (Ck + 1);
   for (int i = threadIdx.x; i < ns; i += blockDim.x) {
     const int c = sl[i];
     atomicOr(&bits[c >> 5], 1u << (c & 31));
-    const int cb = koff[c], len = koff[c + 1] - cb;
-    lex_part += len;
-    if (i < kMaxRanges) { rng_start[i] = cb; rng_cum[i + 1] = len; }
+    const int len = koff[c + 1] - koff[c];
+    lex_part += (len + 7) & ~7;  // padded stream length
+    if (i < kMaxRanges) { rng_start[i] = pof[c]; rng_cum[i + 1] = (len + 7) & ~7; rng_len[i] = len; }
   }
   for (int o = 16; o > 0; o >>= 1) lex_part += __shfl_xor_sync(0xffffffffu, lex_part, o);
   __shared__ long long lex_w[kThreads / 32];
@@ -262,6 +340,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) {
       const uint32_t id_s = tc::idesc_bf16(BQ, BN, false, false);
       const uint32_t id_o = tc::idesc_bf16(BQ, D, false, true);
+      // descriptors are built once; a K step only moves the start-address
+      // field (address >> 4): +2 per 32 B inside a swizzled row, +1024 per
+      // 16 KB region of Q, +16 per 256 B of a K tile, +2*kGroup/16 for V
+      uint64_t qd[2];
+      for (int x = 0; x < 2; ++x) qd[x] = tc::desc_kmajor(tc::smem_u32(smem + S::q_off + x * S::kQTile), BQ * 128u, 0);
+      const uint64_t kd0 = tc::desc_kmajor_g8(tc::smem_u32(smem + S::k_off), kGroup, 0);
+      const uint64_t vd0 = tc::desc_mnmajor_g8(tc::smem_u32(smem + S::v_off), kGroup, 0);
+      constexpr uint64_t kStageStep = (uint64_t)(S::kKTile >> 4);
       bool ok = tc::mbar_wait(q_full, 0, abort_flag, status);
       auto issue_pv = [&](int j) -> bool {
         const int b = j & 1, u0 = ustart(j), np = nparts(j);
@@ -269,12 +355,13 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (!tc::mbar_wait(p_full + x * 2 + b, (j >> 1) & 1, abort_flag, status)) return false;
           tc::tc_fence_after();
           const uint32_t pcol = tmem + kColS + (uint32_t)(x * 128 + b * 64);
+          const uint32_t ocol = tmem + kColO + (uint32_t)x * 128u;
           for (int p = 0; p < np; ++p) {
-            const int st = (u0 + p) % kStages;
-            const uint32_t va = tc::smem_u32(smem + S::v_off + st * S::kKTile);
+            const uint64_t vd = vd0 + (uint64_t)((u0 + p) % kStages) * kStageStep;
+#pragma unroll
             for (int k = 0; k < BN / 16; ++k)
-              tc::mma_ts(tmem + kColO + (uint32_t)x * 128u, pcol + (uint32_t)k * 8u,
-                         tc::desc_mnmajor(va, BN * 128u, k), id_o, (j > 0 || p > 0 || k > 0) ? 1u : 0u);
+              tc::mma_ts(ocol, pcol + (uint32_t)k * 8u, vd + (uint64_t)k * (2u * kGroup >> 4), id_o,
+                         (j > 0 || p > 0 || k > 0) ? 1u : 0u);
           }
           tc::mma_commit(o_done + x * 2 + b);
         }
@@ -289,12 +376,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc::tc_fence_after();
         // S_X[b] was last read as P_X[b] by P.V of tile j-2, issued before
         for (int x = 0; x < ntq; ++x) {
-          const uint32_t qa = tc::smem_u32(smem + S::q_off + x * S::kQTile);
+          const uint32_t scol = tmem + kColS + (uint32_t)(x * 128 + b * 64);
           for (int p = 0; p < np; ++p) {
-            const uint32_t ka = tc::smem_u32(smem + S::k_off + ((u0 + p) % kStages) * S::kKTile);
+            const uint64_t kd = kd0 + (uint64_t)((u0 + p) % kStages) * kStageStep;
+#pragma unroll
             for (int k = 0; k < D / 16; ++k)
-              tc::mma_ss(tmem + kColS + (uint32_t)(x * 128 + b * 64), tc::desc_kmajor(qa, BQ * 128u, k),
-                         tc::desc_kmajor(ka, BN * 128u, k), id_s, (p > 0 || k > 0) ? 1u : 0u);
+              tc::mma_ss(scol, qd[x] + (uint64_t)((k >> 2) * 1024 + (k & 3) * 2), kd + (uint64_t)k * 16u, id_s,
+                         (p > 0 || k > 0) ? 1u : 0u);
           }
           tc::mma_commit(s_full + x * 2 + b);
         }
@@ -323,97 +411,127 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc::mbar_arrive(q_full);
     }
     asm volatile("bar.sync 2, 96;" ::: "memory");  // range prefix ready
-    const bf16* Kh = Kp + (size_t)h * Nk * D;
-    const bf16* Vh = Vp + (size_t)h * Nk * D;
-    const float* LC = lc2 + (size_t)h * Ckpad;
-    const size_t cbase = (size_t)h * Ckpad * D;
-    const int pw = warp - 1;                       // producer warp 0..2
-    const int nstage = ustart(ntile);              // total ring stages of the stream
-    // each producer warp fills every third stage end to end, so up to three
-    // loads are in flight without the warps waiting on one another
-    for (int u = pw; u < nstage; u += 3) {
-      const int st = u % kStages;
-      if (!tc::mbar_wait_warp(kv_empty + st, ((u / kStages) & 1) ^ 1, abort_flag, status)) break;
-      const bool exact = u < n_ex;
-      const int j = exact ? u : n_ex + (u - n_ex) / 2, p = exact ? 0 : (u - n_ex) & 1;
-      int* idx = idx_s + st * BN;
-      float* bias = bias_s + st * BN;
-      if (exact) {
-        // locate key offset j*BN in the concatenated routed ranges
-        const int off0 = j * BN;
-        int ri, ro;
-        if (ns <= kMaxRanges) {
-          int lo = 0, hi = ns;  // largest i with cum[i] <= off0
-          while (hi - lo > 1) {
-            const int mid = (lo + hi) >> 1;
-            if (rng_cum[mid] <= off0) lo = mid; else hi = mid;
+    {
+      // the three producer warps (one per scheduler they share with softmax
+      // warps) build and issue every third stage
+      const int pw = warp - 1;
+      int4* pcs = pieces + pw * 8;  // this warp's piece list
+      const uint8_t* Kh = kpk + (size_t)h * npad * D * 2;
+      const uint8_t* Vh = vpk + (size_t)h * npad * D * 2;
+      const float* LC = lc2 + (size_t)h * Ckpad;
+      const size_t cbase = (size_t)h * Ckpad * D * 2;
+      const int nstage = ustart(ntile);  // total ring stages of the stream
+      const unsigned rot = n_ex > 0 ? (blockIdx.x * 2654435761u + h * 40503u) % (unsigned)n_ex : 0u;
+      for (int u = pw; u < nstage; u += 3) {
+        const int st = u % kStages;
+        if (!tc::mbar_wait_warp(kv_empty + st, ((u / kStages) & 1) ^ 1, abort_flag, status)) break;
+        const bool exact = u < n_ex;
+        int j = exact ? u : n_ex + (u - n_ex) / 2;
+        const int p = exact ? 0 : (u - n_ex) & 1;
+        // blocks start their walk over the routed keys at different tiles (the
+        // softmax does not depend on the order), so that the blocks of a head
+        // do not all read the same popular clusters at the same time
+        if (exact) j = (int)(((unsigned)j + rot) % (unsigned)n_ex);
+        float* bias = bias_s + st * BN;
+        const uint32_t ka = tc::smem_u32(smem + S::k_off + st * S::kKTile);
+        const uint32_t va = tc::smem_u32(smem + S::v_off + st * S::kKTile);
+        if (exact) {
+          // pieces of the padded routed stream in [j*BN, j*BN + BN)
+          int npc = 0, tail = BN;
+          if (lane == 0) {
+            const int pos0 = j * BN, end = pos0 + BN;
+            int ri;
+            if (ns <= kMaxRanges) {
+              int lo = 0, hi = ns;  // largest i with cum[i] <= pos0
+              while (hi - lo > 1) {
+                const int mid = (lo + hi) >> 1;
+                if (rng_cum[mid] <= pos0) lo = mid; else hi = mid;
+              }
+              ri = lo;
+            } else {
+              ri = 0;
+            }
+            int cum = ns <= kMaxRanges ? rng_cum[ri] : 0;
+            int pos = pos0;
+            while (pos < end && ri < ns && npc < 8) {
+              int pst, len;
+              if (ri < kMaxRanges) {
+                pst = rng_start[ri]; len = rng_len[ri];
+              } else {
+                const int c = sl[ri];
+                pst = pof[c]; len = koff[c + 1] - koff[c];
+              }
+              const int plen = (len + 7) & ~7;
+              if (cum + plen <= pos) { cum += plen; ++ri; continue; }  // (ranges past the staged prefix)
+              const int off = pos - cum, take = min(plen - off, end - pos);
+              pcs[npc++] = make_int4((pos - pos0) >> 3, pst + off, take >> 3, max(0, min(len - off, take)));
+              pos += take;
+              cum += plen;
+              ++ri;
+            }
+            tail = pos - pos0;
           }
-          ri = lo; ro = off0 - rng_cum[lo];
+          npc = __shfl_sync(0xffffffffu, npc, 0);
+          tail = __shfl_sync(0xffffffffu, tail, 0);
+          __syncwarp();
+          // bias: valid keys 0, padding and the stream tail -inf
+          for (int i = lane; i < BN; i += 32) bias[i] = -INFINITY;
+          __syncwarp();
+          for (int q = 0; q < npc; ++q) {
+            const int4 pc = pcs[q];
+            for (int i = lane; i < pc.w; i += 32) bias[pc.x * 8 + i] = 0.f;
+          }
+          // zero the rows past the stream end so the MMAs see finite values
+          if (tail < BN) {
+            uint4* kz = reinterpret_cast<uint4*>(smem + S::k_off + st * S::kKTile) + (tail >> 3) * (kGroup / 16);
+            uint4* vz = reinterpret_cast<uint4*>(smem + S::v_off + st * S::kKTile) + (tail >> 3) * (kGroup / 16);
+            const int nz = ((BN - tail) >> 3) * (int)(kGroup / 16);
+            for (int i = lane; i < nz; i += 32) { kz[i] = make_uint4(0, 0, 0, 0); vz[i] = make_uint4(0, 0, 0, 0); }
+            tc::fence_proxy_async();
+          }
+          if (lane == 0) flag_s[st] = 1;
+          __syncwarp();
+          if (lane == 0) {
+            // a piece must stay inside the stage tile and the packed rows;
+            // one that does not is dropped (status word) instead of copied
+            uint32_t okm = 0, bytes = 0;
+            for (int q = 0; q < npc; ++q) {
+              const int4 pc = pcs[q];
+              const bool good = pc.x >= 0 && pc.z > 0 && pc.x + pc.z <= BN / 8 && pc.y >= 0 &&
+                                (size_t)pc.y + (size_t)pc.z * 8 <= npad;
+              if (good) { okm |= 1u << q; bytes += 2u * (uint32_t)pc.z * kGroup; }
+              else set_status(status, ST_BOUNDS);
+            }
+            tc::mbar_arrive_expect_tx(kv_full + st, bytes);
+            for (int q = 0; q < npc; ++q) {
+              if (!((okm >> q) & 1u)) continue;
+              const int4 pc = pcs[q];
+              const uint32_t n = (uint32_t)pc.z * kGroup;
+              const size_t go = (size_t)(pc.y >> 3) * kGroup;
+              tc::bulk_g2s(ka + (uint32_t)pc.x * kGroup, Kh + go, n, kv_full + st);
+              tc::bulk_g2s(va + (uint32_t)pc.x * kGroup, Vh + go, n, kv_full + st);
+            }
+          }
         } else {
-          ri = 0; ro = off0;
-          while (ri < ns) {
-            const int c = sl[ri], len = koff[c + 1] - koff[c];
-            if (ro < len) break;
-            ro -= len; ++ri;
+          const int c0 = (j - n_ex) * BN;
+          for (int i = lane; i < BN; i += 32) {
+            const int c = c0 + i;
+            const bool routed = c < Ck && ((bits[c >> 5] >> (c & 31)) & 1u);
+            bias[i] = routed ? -INFINITY : LC[c];
+          }
+          if (lane == 0) flag_s[st] = 1;
+          __syncwarp();
+          if (lane == 0) {
+            const uint32_t n = (uint32_t)(BN / 8) * kGroup;
+            const size_t go = cbase + (size_t)(c0 >> 3) * kGroup;
+            tc::mbar_arrive_expect_tx(kv_full + st, 2u * n);
+            tc::bulk_g2s(ka, (p == 0 ? kb_hi : kb_lo) + go, n, kv_full + st);
+            tc::bulk_g2s(va, (p == 0 ? vb_hi : vb_lo) + go, n, kv_full + st);
           }
         }
-        int fill = 0;
-        while (fill < BN && ri < ns) {
-          int cb, clen;
-          if (ri < kMaxRanges) {
-            cb = rng_start[ri]; clen = rng_cum[ri + 1] - rng_cum[ri];
-          } else {
-            const int c = sl[ri];
-            cb = koff[c]; clen = koff[c + 1] - cb;
-          }
-          const int take = min(clen - ro, BN - fill);
-          for (int i = lane; i < take; i += 32) idx[fill + i] = cb + ro + i;
-          fill += take;
-          ro += take;
-          if (ro == clen) { ++ri; ro = 0; }
-        }
-        for (int i = fill + lane; i < BN; i += 32) idx[i] = -1;
-        for (int i = lane; i < BN; i += 32) bias[i] = i < fill ? 0.f : -INFINITY;
-        if (lane == 0) flag_s[st] = fill < BN ? 1 : 0;
-      } else {
-        const int c0 = (j - n_ex) * BN;
-        for (int i = lane; i < BN; i += 32) {
-          const int c = c0 + i;
-          idx[i] = c;
-          const bool routed = c < Ck && ((bits[c >> 5] >> (c & 31)) & 1u);
-          bias[i] = routed ? -INFINITY : LC[c];
-        }
-        if (lane == 0) flag_s[st] = 1;
+        __syncwarp();
       }
-      __syncwarp();
-      const uint32_t ka = tc::smem_u32(smem + S::k_off + st * S::kKTile);
-      const uint32_t va = tc::smem_u32(smem + S::v_off + st * S::kKTile);
-      const bf16* ksrc = exact ? Kh : (p == 0 ? kb_hi : kb_lo) + cbase;
-      const bf16* vsrc = exact ? Vh : (p == 0 ? vb_hi : vb_lo) + cbase;
-      {
-        // lane -> (row offset, 16-byte chunk); each warp instruction copies
-        // RPI whole rows (coalesced); row indices are read up front so the
-        // copies issue back to back
-        constexpr int RPI = 32 / CPR, NIT = BN / RPI;
-        const int rofs = lane / CPR, c = lane % CPR;
-        int rows[NIT];
-#pragma unroll
-        for (int i = 0; i < NIT; ++i) rows[i] = idx[i * RPI + rofs];
-#pragma unroll
-        for (int i = 0; i < NIT; ++i) {
-          const int row = rows[i];
-          const uint32_t nb = row >= 0 ? 16u : 0u;
-          const size_t off = (size_t)(row >= 0 ? row : 0) * D + c * 8;
-          const uint32_t so = tc::sw128_offset(i * RPI + rofs, c, BN);
-          tc::cp_async16(ka + so, ksrc + off, nb);
-          tc::cp_async16(va + so, vsrc + off, nb);
-        }
-      }
-      tc::cp_async_wait_all();
-      tc::fence_proxy_async();
-      tc::mbar_arrive(kv_full + st);
     }
-    tc::cp_async_wait_all();
   } else {
     // -------------------------------------------------------------- softmax
     const int x = (warp - 4) >> 2;            // query tile A (0) or B (1)
@@ -546,21 +664,27 @@ __global__ void __launch_bounds__(kThreads, 1)
 int round64(int x) { return (x + 63) / 64 * 64; }
 
 struct AttnWs {
-  bf16 *kh, *kl, *vh, *vl;
+  uint8_t *kh, *kl, *vh, *vl, *kpk, *vpk;
+  int32_t* poff;
   float* lc2;
   int2* tiles;
   int32_t* ntiles;
+  size_t npad;
 };
 
-size_t attn_layout(int H, int Nq, int d, int Cq, int Ck, AttnWs* out, void* ws) {
+size_t attn_layout(int H, int Nq, int Nk, int d, int Cq, int Ck, AttnWs* out, void* ws) {
   Carve cv(ws);
   const int Ckpad = round64(Ck);
   const int tmax = (Nq + kUnitRows - 1) / kUnitRows + Cq;
   AttnWs w;
-  w.kh = cv.take<bf16>((size_t)H * Ckpad * d);
-  w.kl = cv.take<bf16>((size_t)H * Ckpad * d);
-  w.vh = cv.take<bf16>((size_t)H * Ckpad * d);
-  w.vl = cv.take<bf16>((size_t)H * Ckpad * d);
+  w.npad = (size_t)Nk + 8 * (size_t)Ck;  // rows after padding every cluster to 8
+  w.kh = cv.take<uint8_t>((size_t)H * Ckpad * d * 2);
+  w.kl = cv.take<uint8_t>((size_t)H * Ckpad * d * 2);
+  w.vh = cv.take<uint8_t>((size_t)H * Ckpad * d * 2);
+  w.vl = cv.take<uint8_t>((size_t)H * Ckpad * d * 2);
+  w.kpk = cv.take<uint8_t>((size_t)H * w.npad * d * 2);
+  w.vpk = cv.take<uint8_t>((size_t)H * w.npad * d * 2);
+  w.poff = cv.take<int32_t>((size_t)H * (Ck + 1));
   w.lc2 = cv.take<float>((size_t)H * Ckpad);
   w.tiles = cv.take<int2>((size_t)H * tmax);
   w.ntiles = cv.take<int32_t>(H);
@@ -574,18 +698,22 @@ cudaError_t launch(const void* Qp, const void* Kp, const void* Vp, const int32_t
                    const int32_t* n_sel, int H, int Nq, int Nk, int Cq, int Ck, float scale, void* O,
                    void* ws, cudaStream_t st) {
   AttnWs w;
-  attn_layout(H, Nq, D, Cq, Ck, &w, ws);
+  attn_layout(H, Nq, Nk, D, Cq, Ck, &w, ws);
   const int Ckpad = round64(Ck);
   const int tmax = (Nq + kUnitRows - 1) / kUnitRows + Cq;
   k_prep_comp<D><<<dim3(Ckpad, H), 64, 0, st>>>(Kbar, Vbar, k_off, Ck, Ckpad, w.kh, w.kl, w.vh, w.vl, w.lc2);
+  note_launch();
+  k_pad_offsets<<<H, 1024, 0, st>>>(k_off, Ck, w.poff); note_launch();
+  k_pack<D><<<dim3(Ck, H), 256, 0, st>>>(static_cast<const bf16*>(Kp), static_cast<const bf16*>(Vp), k_off, w.poff,
+                                         Nk, Ck, w.npad, w.kpk, w.vpk);
   note_launch();
   k_tile_table_tc<<<H, 1024, 0, st>>>(q_off, Cq, tmax, w.tiles, w.ntiles); note_launch();
   const int smem = AttnSmem<D>::total;
   cudaError_t e = cudaFuncSetAttribute(k_attn_tc<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
   k_attn_tc<D><<<dim3(tmax, H), kThreads, smem, st>>>(
-      static_cast<const bf16*>(Qp), static_cast<const bf16*>(Kp), static_cast<const bf16*>(Vp), q_off, k_off,
-      perm_q, w.kh, w.kl, w.vh, w.vl, w.lc2, sel, n_sel, w.tiles, w.ntiles, tmax, Nq, Nk, Cq, Ck, Ckpad, scale * kLog2e,
+      static_cast<const bf16*>(Qp), w.kpk, w.vpk, w.npad, q_off, k_off, w.poff, perm_q, w.kh, w.kl, w.vh, w.vl,
+      w.lc2, sel, n_sel, w.tiles, w.ntiles, tmax, Nq, Nk, Cq, Ck, Ckpad, scale * kLog2e,
       static_cast<bf16*>(O), status_word());
   note_launch();
   return cudaGetLastError();
@@ -595,9 +723,9 @@ cudaError_t launch(const void* Qp, const void* Kp, const void* Vp, const int32_t
 
 bool attn_tc_supported(int d, int Ck) { return (d == 64 || d == 128) && Ck <= kMaxCkBits; }
 
-size_t attn_tc_ws_bytes(int H, int Nq, int d, int Cq, int Ck) {
+size_t attn_tc_ws_bytes(int H, int Nq, int Nk, int d, int Cq, int Ck) {
   if (!attn_tc_supported(d, Ck)) return 0;
-  return attn_layout(H, Nq, d, Cq, Ck, nullptr, nullptr);
+  return attn_layout(H, Nq, Nk, d, Cq, Ck, nullptr, nullptr);
 }
 
 cudaError_t attn_tc_run(const void* Qp, const void* Kp, const void* Vp, const int32_t* q_off,

@@ -7,7 +7,7 @@
 namespace svg {
 constexpr int kMaxCkBits = 4096;
 bool attn_tc_supported(int d, int Ck);
-size_t attn_tc_ws_bytes(int H, int Nq, int d, int Cq, int Ck);
+size_t attn_tc_ws_bytes(int H, int Nq, int Nk, int d, int Cq, int Ck);
 cudaError_t attn_tc_run(const void* Qp, const void* Kp, const void* Vp, const int32_t* q_off,
                         const int32_t* k_off, const int32_t* perm_q, const float* Kbar,
                         const float* Vbar, const int32_t* sel, const int32_t* n_sel, int H, int Nq,

@@ -46,7 +46,7 @@ cudaError_t route_run(const float* E, const int32_t* k_counts, const int32_t* q_
                       int32_t* n_sel, int64_t* exec_pairs, cudaStream_t st);
 
 // ---- hybrid attention
-size_t attn_ws_bytes(int H, int Nq, int d, int Cq, int Ck);
+size_t attn_ws_bytes(int H, int Nq, int Nk, int d, int Cq, int Ck);
 cudaError_t attn_run(const void* Qp, const void* Kp, const void* Vp, const int32_t* q_off,
                      const int32_t* k_off, const int32_t* perm_q, const float* Kbar,
                      const float* Vbar, const int32_t* sel, const int32_t* n_sel, int dtype,

@@ -78,6 +78,12 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
   }
 }
 
+// Arrive once and add `bytes` to the transaction count of the current phase.
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
+               : "memory");
+}
+
 // mbar_wait for code that follows with warp-collective (.sync.aligned)
 // instructions: the result is made uniform across the warp, so that either
 // every lane goes on or every lane takes the abort path.
@@ -198,6 +204,18 @@ __device__ __forceinline__ uint64_t desc_mnmajor(uint32_t tile_saddr, uint32_t r
   return sdesc(tile_saddr + (uint32_t)k16 * 2048u, region_bytes, 1024, kSwizzle128);
 }
 
+// Operands in the "8-row group" layout (no swizzle): groups of 8 rows stored
+// as [16-byte chunk][row][16 B], group_bytes = 8 * row_bytes apart.  The
+// 8 x 16 B core matrices are contiguous, so the same bytes are a canonical
+// K-major operand when rows are the M/N dimension ...
+__device__ __forceinline__ uint64_t desc_kmajor_g8(uint32_t tile_saddr, uint32_t group_bytes, int k16) {
+  return sdesc(tile_saddr + (uint32_t)k16 * 256u, 128u, group_bytes, 0u);
+}
+// ... and a canonical MN-major operand when rows are the K dimension.
+__device__ __forceinline__ uint64_t desc_mnmajor_g8(uint32_t tile_saddr, uint32_t group_bytes, int k16) {
+  return sdesc(tile_saddr + (uint32_t)k16 * 2u * group_bytes, group_bytes, 128u, 0u);
+}
+
 // Instruction descriptor, kind::f16 with bf16 A/B and f32 accumulation.
 __host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, bool a_mn_major, bool b_mn_major) {
   return (1u << 4) | (1u << 7) | (1u << 10) | ((a_mn_major ? 1u : 0u) << 15) |
@@ -232,6 +250,15 @@ __device__ __forceinline__ void mma_commit(uint64_t* bar) {
 }
 
 // ------------------------------------------------- cp.async row copies
+
+// Bulk global -> shared copy of `bytes` (multiple of 16, both addresses
+// 16-byte aligned) completing as transaction bytes on `bar`.
+__device__ __forceinline__ void bulk_g2s(uint32_t dst, const void* src, uint32_t bytes, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
+      "l"(src), "r"(bytes), "r"(smem_u32(bar))
+      : "memory");
+}
 
 // 16-byte global -> shared copy; src_bytes = 0 fills zeros.
 __device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, uint32_t src_bytes) {
