@@ -58,6 +58,12 @@ int check_params(const svgear_params* p) {
   return SVGEAR_OK;
 }
 
+}  // namespace
+
+int params_status(const svgear_params* p) { return check_params(p); }
+
+namespace {
+
 float eff_scale(const svgear_params* p) {
   return p->scale > 0.f ? p->scale : 1.0f / std::sqrt((float)p->d);
 }

@@ -13,6 +13,9 @@
 // This is exact algebra; the form keeps full relative accuracy when the
 // cluster is tight (u -> 0, v -> vbar) where a^2|vbar|^2 - 2ab vbar.v + b^2|v|^2
 // would cancel.  Logits never leave registers.
+#include <mutex>
+
+#include "../../include/svgear.h"
 #include "common.cuh"
 #include "internal.h"
 
@@ -151,4 +154,51 @@ cudaError_t block_error_run(const float* Qbar, const float* Kbar, const float* V
   return cudaGetLastError();
 }
 
+// ---------------------------------------------------------------------------
+// Allocation-free variant: the centroid-logit scratch lives in a file-scope
+// device array instead of a caller workspace.  Every GPU that loads the
+// library holds this array until the process exits.
+constexpr size_t kNoAllocScratchFloats = size_t(1) << 21;  // 8 MiB: H*Cq*Ck <= 2,097,152
+static __device__ __align__(256) float g_noalloc_scratch[kNoAllocScratchFloats];
+
+// Device address of g_noalloc_scratch on the current device, looked up once
+// per device (the symbol name is only a host-side handle).
+static float* noalloc_scratch(cudaError_t* err) {
+  static std::mutex mu;
+  static float* cache[64] = {nullptr};
+  int dev = 0;
+  *err = cudaGetDevice(&dev);
+  if (*err != cudaSuccess) return nullptr;
+  if (dev < 0 || dev >= 64) { *err = cudaErrorInvalidDevice; return nullptr; }
+  std::lock_guard<std::mutex> lock(mu);
+  if (!cache[dev]) {
+    void* ptr = nullptr;
+    *err = cudaGetSymbolAddress(&ptr, g_noalloc_scratch);
+    if (*err != cudaSuccess) return nullptr;
+    cache[dev] = static_cast<float*>(ptr);
+  }
+  return cache[dev];
+}
+
 }  // namespace svg
+
+extern "C" int svgear_block_error_noalloc(const float* Qbar, const float* Kbar, const float* Vbar,
+                                          const void* Kp, const void* Vp, const int32_t* k_off,
+                                          const float* key_scalars, const svgear_params* p, float* E,
+                                          float* M, void* stream) {
+  using namespace svg;
+  const int r = params_status(p);
+  if (r != SVGEAR_OK) return r;
+  if (!Qbar || !Kbar || !Kp || !k_off || !key_scalars || !E || !M) return SVGEAR_ERR_INVALID;
+  const uintptr_t mis = reinterpret_cast<uintptr_t>(Qbar) | reinterpret_cast<uintptr_t>(Kbar) |
+                        reinterpret_cast<uintptr_t>(Kp);
+  if (mis & 15u) return SVGEAR_ERR_INVALID;
+  if ((size_t)p->H * (size_t)p->Cq * (size_t)p->Ck > kNoAllocScratchFloats) return SVGEAR_ERR_WORKSPACE;
+  cudaError_t e = cudaSuccess;
+  float* L = noalloc_scratch(&e);
+  if (!L) return SVGEAR_ERR_CUDA;
+  const float scale = p->scale > 0.f ? p->scale : 1.0f / sqrtf((float)p->d);
+  e = block_error_run(Qbar, Kbar, Vbar, Kp, Vp, k_off, key_scalars, p->dtype, p->H, p->Nk, p->d, p->Cq,
+                      p->Ck, scale, E, M, L, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? SVGEAR_OK : SVGEAR_ERR_CUDA;
+}

@@ -5,6 +5,8 @@
 #include <stddef.h>
 #include <stdint.h>
 
+#include "../../include/svgear.h"
+
 namespace svg {
 
 // Device status word of the current device (see svgear_get_status).
@@ -12,6 +14,9 @@ int* status_word();
 
 // Counts kernel launches issued by the library (svgear_launch_count).
 void note_launch();
+
+// Host-side validation of an operator parameter block (svgear_status code).
+int params_status(const svgear_params* p);
 
 // ---- stable counting sort of labels (shared by k-means update and permute)
 // chunk = tokens per scatter chunk; nchunk = ceil(N / chunk)

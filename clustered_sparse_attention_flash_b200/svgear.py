@@ -76,6 +76,7 @@ _SIGS = {
     "svgear_permute": (_I, [_P, _I, _P, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P, _P, _P, _SZ, _P]),
     "svgear_block_error_workspace_size": (_SZ, [_PP]),
     "svgear_block_error": (_I, [_P, _P, _P, _P, _P, _P, _P, _PP, _P, _P, _P, _SZ, _P]),
+    "svgear_block_error_noalloc": (_I, [_P, _P, _P, _P, _P, _P, _P, _PP, _P, _P, _P]),
     "svgear_route": (_I, [_P, _P, _P, _PP, _P, _P, _P, _P, _P]),
     "svgear_hybrid_attn_workspace_size": (_SZ, [_PP]),
     "svgear_hybrid_attn": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _PP, _P, _P, _SZ, _P]),
@@ -192,6 +193,12 @@ def svgear_block_error(Qbar, Kbar, Vbar, Kp, Vp, k_off, key_scalars, p, E, M, ws
     _check("svgear_block_error", lib().svgear_block_error(
         _ptr(Qbar), _ptr(Kbar), _ptr(Vbar), _ptr(Kp), _ptr(Vp), _ptr(k_off), _ptr(key_scalars),
         ctypes.byref(p), _ptr(E), _ptr(M), _ptr(ws), ws_bytes, _stream(stream)))
+
+
+def svgear_block_error_noalloc(Qbar, Kbar, Vbar, Kp, Vp, k_off, key_scalars, p, E, M, stream=None):
+    _check("svgear_block_error_noalloc", lib().svgear_block_error_noalloc(
+        _ptr(Qbar), _ptr(Kbar), _ptr(Vbar), _ptr(Kp), _ptr(Vp), _ptr(k_off), _ptr(key_scalars),
+        ctypes.byref(p), _ptr(E), _ptr(M), _stream(stream)))
 
 
 def svgear_route(E, k_counts, q_counts, p, mask, sel, n_sel, exec_pairs, stream=None):

@@ -171,6 +171,33 @@ SVGEAR_API int svgear_block_error(const float* Qbar, const float* Kbar, const fl
                        float* E, float* M, void* ws, size_t ws_bytes, void* stream);
 
 /* ---------------------------------------------------------------------------
+ * svgear_block_error without a workspace argument.  No counterpart in the
+ * paper: this entry point exists for callers that cannot allocate device
+ * memory at the point of the call -- for example a runtime that plans all of
+ * its device memory ahead of time and hands the operator only its inputs and
+ * outputs, or a plug-in running inside a host framework that owns the device
+ * allocator and exposes none of it.
+ * Same arguments, results and errors as svgear_block_error, except:
+ *   - the scratch buffer is a file-scope device array of this library of
+ *     2,097,152 floats (8 MiB), held on every GPU that loads the library
+ *     until the process exits; H * Cq * Ck above that limit returns
+ *     SVGEAR_ERR_WORKSPACE without enqueuing anything;
+ *   - the first call on a device looks up the array's device address
+ *     (cudaGetSymbolAddress) with that device current; make that first call
+ *     before any stream capture;
+ *   - every call shares the one array, so calls that overlap on the GPU
+ *     (different streams, or different host threads on one device) race and
+ *     must be ordered by the caller.  Each call writes the scratch fully
+ *     before reading it, so nothing carries over between calls.
+ * It calls no device allocator (cudaMalloc, cudaFree or a library that
+ * allocates).
+ * ------------------------------------------------------------------------- */
+SVGEAR_API int svgear_block_error_noalloc(const float* Qbar, const float* Kbar, const float* Vbar,
+                       const void* Kp, const void* Vp, const int32_t* k_off,
+                       const float* key_scalars, const svgear_params* p,
+                       float* E, float* M, void* stream);
+
+/* ---------------------------------------------------------------------------
  * (3) Error-aware routing.  Review step (3); gist.science 2.B "Selektion".
  * Per (h, a): non-empty key clusters in E-descending order (equal E: smaller
  * c first); the longest prefix whose total size fits floor(rho*Nk) is routed
