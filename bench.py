@@ -44,6 +44,8 @@ def _args():
     ap.add_argument("--rho", type=float, default=None)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--heads", type=int, default=None,
+                    help="run only the first H heads of the workload (small profiler captures)")
     return ap.parse_args()
 
 
@@ -140,6 +142,30 @@ def _peaks():
         return 1400.0, 6650.0, "fallback"
 
 
+# DRAM traffic of the attention kernel from one ncu capture (dram__bytes_read.sum
+# + dram__bytes_write.sum of k_attn_tc on the first 4 heads of the Wan-shaped
+# workload: 345.5 MB, i.e. 86.4 MB per head; traffic grows with the heads).  The
+# figure holds only for the kernel sources it was taken on, identified by hash.
+_ATTN_TRAFFIC = {"bytes_per_head": 345.5e6 / 4, "workload": "wan",
+                 "sources": ("attn_tc.cu", "attn_tc.cuh", "tc_common.cuh"),
+                 "sha1": "5fdd31828da8cb2c8124a5982d6717bc21d423de"}
+
+
+def attn_traffic(cfg):
+    """Per-launch DRAM bytes of k_attn_tc, or None when the capture does not
+    apply (another workload, or kernel sources changed since)."""
+    import hashlib
+    if cfg.name != _ATTN_TRAFFIC["workload"]:
+        return None
+    h = hashlib.sha1()
+    for f in _ATTN_TRAFFIC["sources"]:
+        with open(os.path.join(ROOT, "clustered_sparse_attention_flash_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    if h.hexdigest() != _ATTN_TRAFFIC["sha1"]:
+        return None
+    return _ATTN_TRAFFIC["bytes_per_head"] * cfg.H
+
+
 # ----------------------------------------------------------------- oracle
 
 def oracle_sample(cfg, rho, q, k, v, iq, ik):
@@ -233,6 +259,8 @@ def main():
     a = _args()
     from clustered_sparse_attention_flash_b200 import synth
     cfg = synth.CONFIGS[a.config]
+    if a.heads is not None:
+        cfg = cfg.with_(H=a.heads)
     rho = cfg.rho if a.rho is None else a.rho
     if a.impl == "reference":
         return run_reference(a, cfg, rho)
@@ -344,9 +372,10 @@ def main():
     achieved = attn_flops / (avg["ms_attn"] / 1e3) / 1e12
     roofline = {"kernel": "hybrid attention (svgear_hybrid_attn)", "bound": "tensor",
                 "achieved": achieved, "peak": peak_tc, "unit": "TFLOP/s", "frac": achieved / peak_tc,
-                "traffic": None,
+                "traffic": attn_traffic(cfg),
                 "note": f"algorithmic 4*d*(executed + compensated pairs) per launch over the stage's "
-                        f"CUDA-event time; peak = {peak_src} sustained dense bf16"}
+                        f"CUDA-event time; peak = {peak_src} sustained dense bf16; traffic = DRAM "
+                        f"bytes per launch from an ncu capture of 4 heads, scaled by heads"}
 
     cpu = None
     if rank == 0 and world == 1 and not a.no_cpu_baseline:
