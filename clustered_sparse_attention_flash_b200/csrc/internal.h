@@ -58,6 +58,15 @@ cudaError_t attn_run(const void* Qp, const void* Kp, const void* Vp, const int32
                      int H, int Nq, int Nk, int d, int Cq, int Ck, float scale, void* O,
                      void* ws, cudaStream_t st);
 
+// ---- TMA tensor maps (tma_host.cu)
+constexpr int kTmaMapBytes = 128;
+bool tma_available();
+// Tiled map of a bf16 tensor [d2][d1][d0] (d0 contiguous) with box
+// {64, box1, 1} and 128-byte swizzle, written to `map` (kTmaMapBytes bytes,
+// 64-byte aligned).  Out-of-range rows read as zeros.  False when the driver
+// entry point is missing or the arguments are not encodable.
+bool tma_map_bf16_3d(void* map, const void* base, uint64_t d0, uint64_t d1, uint64_t d2, uint32_t box1);
+
 inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
 // Bump allocator over a caller-provided workspace.

@@ -172,7 +172,7 @@ cudaError_t kmeans_run(const void* X, int dtype, int H, int N, int d, int C, int
   if (offsets_out) offs = offsets_out;
   if (dtype == DT_BF16) {
     const bf16* x = static_cast<const bf16*>(X);
-    const bool tc = kmeans_tc_supported(d, C);
+    const bool tc = kmeans_tc_usable(X, N, d, C);
     if (d == 128) return run_t<bf16, 128>(x, H, N, C, iters, init, cent, labels, counts, offs, perm, sws, tws, tc, st);
     return run_t<bf16, 64>(x, H, N, C, iters, init, cent, labels, counts, offs, perm, sws, tws, tc, st);
   }

@@ -1,25 +1,34 @@
 // Tensor-core k-means assignment for bf16 tokens (SVG-EAR review, step (1):
 // "Flash k-means" clustering of queries and keys).
 //
-// For a tile of 128 tokens the scores x . mu_c of every centroid come from
-// tcgen05 MMAs (A = token tile, B = bf16-rounded centroids resident in shared
-// memory, fp32 accumulators in tensor memory).  The epilogue forms
-// s_c = ||mu_c||^2 - 2 x.mu_c and keeps, per token, the running minimum and
-// every centroid whose score lies within 2B of it, where B bounds the score
-// error: rounding the centroid to bf16 moves x.mu by at most ||x|| ||mu - bf16(mu)||,
-// the fp32 accumulation by at most 2^-14 ||x|| ||bf16(mu)||, plus the
-// rounding of ||mu||^2 and of the epilogue FMA.  A single survivor is the exact
-// argmin; otherwise the token goes on a list that k_refine re-decides with
-// float64 distances (smaller index on equal distance), so labels equal the
-// exact argmin.
+// The nearest centroid of x is the one with the largest score
+//   s_c = x . mu_c - ||mu_c||^2 / 2.
+// For a tile of 128 tokens, x . mu_c comes from tcgen05 MMAs (A = token tile,
+// B = bf16-rounded centroids resident in shared memory, fp32 accumulators in
+// tensor memory, 128 centroid columns per accumulator slot).  The epilogue
+// subtracts ||mu_c||^2 / 2, writes the column index into the low mantissa bits
+// of the score (so one float carries score and index, and no two columns tie)
+// and keeps the three largest packed scores b1 >= b2 >= b3 per token.
 //
-// Block of 12 warps: warp 0 allocates tensor memory and issues MMAs, warps 1-3
-// copy tiles (cp.async into the 128-byte-swizzled layout), warps 4-7 and 8-11
-// are two epilogue warpgroups that take alternate 256-column accumulator slots.
-// The epilogue reads each slot twice: a branch-free minimum pass, then a pass
-// that lists every column inside the window of the minimum.
+// Every packed score is within E of the exact s_c (bf16 rounding of mu, the
+// fp32 accumulation inside the MMA, the subtraction, the index bits; bound
+// below), so the exact best column has a packed score >= b1 - 2E:
+//   b2 <  b1 - 2E            -> the label is the column of b1 (exact);
+//   b3 <  b1 - 2E <= b2      -> one of the columns of b1, b2: decided in float64;
+//   otherwise                -> every centroid is checked in float64.
+// Ties in float64 go to the smaller index, so labels equal the exact argmin.
+//
+// Block of 10 warps: warp 0 allocates tensor memory and issues MMAs, warp 1
+// issues the TMA copies (centroid table once, token tiles through a ring of
+// stages), warps 2-5 and 6-9 are two epilogue warpgroups that take alternate
+// 128-column chunks.  When a tile has chunks in both warpgroups, the one that
+// did not see the tile's last chunk hands its partial top three to the other
+// through shared memory (mbarrier-synchronised, no lockstep).
+#include <cuda.h>
+
 #include <algorithm>
 #include <cfloat>
+#include <climits>
 
 #include "internal.h"
 #include "kmeans_tc.cuh"
@@ -29,38 +38,58 @@ namespace svg {
 
 namespace {
 
-constexpr int BM = 128;
-constexpr int KC = 6;                     // candidate list capacity per token
-constexpr int kThreads = 384;
-constexpr int kProducers = 96;
-constexpr int kCentBytesMax = 128 * 1024;
-constexpr int kSlotCols = 256;
-constexpr int kRefineInts = 4 + KC;   // h, row, n (-1 = overflow), pad, candidates
+constexpr int BM = 128;                // tokens per tile (MMA M)
+constexpr int kThreads = 320;
+constexpr int kChunk = 128;            // accumulator columns per TMEM slot
+constexpr int kSlots = 4;
+constexpr int kMaxStages = 6;
+constexpr int kRefineInts = 8;         // h, row, n (2, or -1 = all centroids), c1, c2, pad
+constexpr int kSmemLimit = 232448;     // opt-in dynamic shared memory per block
+constexpr int kMaxC = 1024;            // index bits packed into the score: at most 10
+constexpr float kPadHalfNorm = 1e30f;  // ||mu||^2/2 of padding columns: never best, finite
 
 __host__ __device__ inline int round16(int x) { return (x + 15) & ~15; }
+__host__ __device__ inline int round128(int x) { return (x + 127) & ~127; }
 
-struct Bounds {  // per head
+struct Bounds {  // per head; non-negative floats, combined with integer atomicMax
   float dmax;    // max_c ||mu_c - bf16(mu_c)||
   float mmax;    // max_c ||bf16(mu_c)||
   float nmax;    // max_c ||mu_c||^2
-  float pad;
+  int pad;
 };
 
-// Per head: bf16 copy of the centroids (zero rows up to Cpad), ||mu||^2
-// (+inf on padding rows) and the error-bound maxima.
+// Shared-memory layout of the assignment kernel (offsets from a 1024-aligned base).
+struct Lay {
+  int cent, x, tab, merge, bars, total;
+};
+__host__ __device__ inline Lay layout(int D, int Cr, int Cpad, int stages) {
+  Lay l;
+  l.cent = 0;
+  l.x = Cr * D * 2;                          // Cr is a multiple of 128: 1024-aligned
+  l.tab = l.x + stages * BM * D * 2;
+  l.merge = l.tab + Cpad * 8;
+  l.bars = l.merge + 2 * 3 * BM * 4;
+  l.total = l.bars + 32 * 8 + 1024;          // barriers, TMEM slot, abort flag; alignment slack
+  return l;
+}
+
+// Per centroid row (one warp each): bf16 copy (zero rows up to Cr), the table
+// entry {||mu||^2 / 2, index} (padding columns up to Cpad get kPadHalfNorm) and
+// the per-head maxima of the error bound.
 template <int D>
-__global__ void __launch_bounds__(256) k_prep_centroids(const float* __restrict__ cent, int C, int Cpad,
-                                                        bf16* __restrict__ cb, float* __restrict__ cnorm,
+__global__ void __launch_bounds__(256) k_prep_centroids(const float* __restrict__ cent, int C, int Cpad, int Cr,
+                                                        bf16* __restrict__ cb, int2* __restrict__ table,
                                                         Bounds* __restrict__ bounds) {
   __shared__ float red[3][8];
-  const int h = blockIdx.x, w = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int h = blockIdx.y, w = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int c = blockIdx.x * 8 + w;
   float dmax = 0.f, mmax = 0.f, nmax = 0.f;
-  for (int c = w; c < Cpad; c += 8) {
+  if (c < Cr) {
     double dn = 0.0, mb = 0.0, n2 = 0.0;
     for (int t = lane; t < D; t += 32) {
       const float m = c < C ? cent[((size_t)h * C + c) * D + t] : 0.f;
       const bf16 b = __float2bfloat16_rn(m);
-      cb[((size_t)h * Cpad + c) * D + t] = b;
+      cb[((size_t)h * Cr + c) * D + t] = b;
       const double bd = (double)__bfloat162float(b);
       dn += ((double)m - bd) * ((double)m - bd);
       mb += bd * bd;
@@ -71,199 +100,203 @@ __global__ void __launch_bounds__(256) k_prep_centroids(const float* __restrict_
       mb += __shfl_xor_sync(0xffffffffu, mb, o);
       n2 += __shfl_xor_sync(0xffffffffu, n2, o);
     }
-    if (lane == 0) cnorm[(size_t)h * Cpad + c] = c < C ? (float)n2 : INFINITY;
+    if (lane == 0 && c < Cpad)
+      table[(size_t)h * Cpad + c] = make_int2(__float_as_int(c < C ? (float)(0.5 * n2) : kPadHalfNorm), c);
     if (c < C) {
-      dmax = fmaxf(dmax, (float)sqrt(dn));
-      mmax = fmaxf(mmax, (float)sqrt(mb));
-      nmax = fmaxf(nmax, (float)n2);
+      dmax = (float)sqrt(dn);
+      mmax = (float)sqrt(mb);
+      nmax = (float)n2;
     }
   }
   if (lane == 0) { red[0][w] = dmax; red[1][w] = mmax; red[2][w] = nmax; }
   __syncthreads();
-  if (threadIdx.x == 0) {
-    Bounds b{0.f, 0.f, 0.f, 0.f};
-    for (int i = 0; i < 8; ++i) {
-      b.dmax = fmaxf(b.dmax, red[0][i]);
-      b.mmax = fmaxf(b.mmax, red[1][i]);
-      b.nmax = fmaxf(b.nmax, red[2][i]);
-    }
-    // round the maxima up a little so the bound stays an upper bound
-    b.dmax *= 1.0001f; b.mmax *= 1.0001f; b.nmax *= 1.0001f;
-    bounds[h] = b;
+  if (threadIdx.x < 3) {
+    float m = 0.f;
+    for (int i = 0; i < 8; ++i) m = fmaxf(m, red[threadIdx.x][i]);
+    // rounded up a little so that the bound stays an upper bound
+    atomicMax(reinterpret_cast<int*>(&bounds[h]) + threadIdx.x, __float_as_int(m * 1.0001f));
   }
 }
 
-// ||x_i|| per token (float, rounded up slightly), once per k-means call.
+// ||x_i|| per token (float, rounded up slightly), once per k-means call: D/8
+// lanes per row, 16-byte loads.
 template <int D>
-__global__ void k_row_norms(const bf16* __restrict__ X, long long rows, float* __restrict__ xn) {
-  const long long r = (long long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
-  if (r >= rows) return;
+__global__ void __launch_bounds__(256) k_row_norms(const bf16* __restrict__ X, long long rows,
+                                                   float* __restrict__ xn) {
+  constexpr int LPR = D / 8, RPW = 32 / LPR;
   const int lane = threadIdx.x & 31;
-  float s = 0.f;
-  for (int t = lane * 2; t < D; t += 64) {
-    const float2 v = ld2(X + r * D + t);
-    s = fmaf(v.x, v.x, fmaf(v.y, v.y, s));
-  }
-  for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
-  if (lane == 0) xn[r] = sqrtf(s) * 1.00001f;
-}
-
-// Per-token candidate state: minimum score, number of listed candidates and
-// an overflow flag in registers; the list (KC entries per epilogue thread,
-// strided by the 256 epilogue threads) in shared memory.
-struct Cands {
-  float best;
-  int n;
-  int over;
-};
-
-// Drop listed candidates that fell out of the window after `best` decreased.
-__device__ __forceinline__ void cand_compact(Cands& st, float W, float* ls, int* lc) {
-  int m = 0;
-  for (int i = 0; i < min(st.n, KC); ++i) {
-    const float v = ls[i * 256];
-    if (v <= st.best + W) { ls[m * 256] = v; lc[m * 256] = lc[i * 256]; ++m; }
-  }
-  st.n = m;
-}
-
-__device__ __forceinline__ void cand_push(Cands& st, float s, int c, float* ls, int* lc) {
-  if (st.n < KC) { ls[st.n * 256] = s; lc[st.n * 256] = c; }
-  else st.over = 1;
-  ++st.n;
-}
-
-// Pass 1: minimum score over 32 columns (branch-free).
-__device__ __forceinline__ float min32(const uint32_t (&v)[32], const float* cn) {
-  float m = INFINITY;
+  const long long nw = (long long)gridDim.x * (blockDim.x >> 5);
+  for (long long r0 = ((long long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5)) * RPW; r0 < rows;
+       r0 += nw * RPW) {
+    const long long r = r0 + lane / LPR;
+    float s = 0.f;
+    if (r < rows) {
+      const uint4 u = *reinterpret_cast<const uint4*>(X + r * D + (lane % LPR) * 8);
+      const uint32_t w4[4] = {u.x, u.y, u.z, u.w};
 #pragma unroll
-  for (int q = 0; q < 32; q += 4) {
-    const float4 n4 = *reinterpret_cast<const float4*>(cn + q);
-    const float a = fmaf(-2.f, __uint_as_float(v[q]), n4.x), b = fmaf(-2.f, __uint_as_float(v[q + 1]), n4.y);
-    const float c = fmaf(-2.f, __uint_as_float(v[q + 2]), n4.z), d = fmaf(-2.f, __uint_as_float(v[q + 3]), n4.w);
-    m = fminf(m, fminf(fminf(a, b), fminf(c, d)));
-  }
-  return m;
-}
-
-// Pass 2: list every column whose score is within the fixed threshold.
-template <int G>
-__device__ __forceinline__ void collect(Cands& st, const uint32_t (&v)[G], const float* cn, int cbase, int C,
-                                        float thr, float* ls, int* lc) {
+      for (int i = 0; i < 4; ++i) {
+        const float a = __uint_as_float(w4[i] << 16), b = __uint_as_float(w4[i] & 0xffff0000u);
+        s = fmaf(a, a, fmaf(b, b, s));
+      }
+    }
 #pragma unroll
-  for (int q = 0; q < G; ++q) {
-    const float sq = fmaf(-2.f, __uint_as_float(v[q]), cn[q]);
-    if (sq <= thr && cbase + q < C) cand_push(st, sq, cbase + q, ls, lc);
+    for (int o = LPR / 2; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+    if (r < rows && lane % LPR == 0) xn[r] = sqrtf(s) * 1.00001f;
   }
 }
 
-// Rows the tensor-core pass left ambiguous: one warp per row computes float64
-// distances ||x - mu_c||^2 to each listed candidate (to every centroid when
-// the list overflowed) and keeps the smallest (smaller index on ties).
+// Rows the tensor-core pass left ambiguous, one warp each: float64 distances
+// ||x - mu_c||^2 to the two listed candidates (lanes split the dimensions), or
+// to every centroid (lanes split the centroids); the smallest wins, the
+// smaller index on ties.
 template <int D>
 __global__ void __launch_bounds__(256) k_refine(const bf16* __restrict__ X, const float* __restrict__ cent,
                                                 int N, int C, const int* __restrict__ refine,
                                                 const int* __restrict__ count, int32_t* __restrict__ labels) {
   constexpr int PER = D / 32;
-  const int lane = threadIdx.x & 31;
+  __shared__ float xs[8][D];
+  const int lane = threadIdx.x & 31, wib = threadIdx.x >> 5;
   const int nw = gridDim.x * (blockDim.x >> 5);
   const int total = *count;
-  for (int w = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); w < total; w += nw) {
+  for (int w = blockIdx.x * (blockDim.x >> 5) + wib; w < total; w += nw) {
     const int* e = refine + (size_t)w * kRefineInts;
     const int h = e[0], row = e[1], n = e[2];
-    float xv[PER];
-    {
-      const bf16* xr = X + ((size_t)h * N + row) * D + lane * PER;
-      if constexpr (PER == 4) {
-        const float4 v = ld4(xr);
-        xv[0] = v.x; xv[1] = v.y; xv[2] = v.z; xv[3] = v.w;
-      } else {
-        const float2 v = ld2(xr);
-        xv[0] = v.x; xv[1] = v.y;
-      }
-    }
-    const int cnt = n < 0 ? C : n;
-    double best = 1e300;
-    int bc = 0;
-    for (int i = 0; i < cnt; ++i) {
-      const int c = n < 0 ? i : e[3 + i];
-      const float* mu = cent + ((size_t)h * C + c) * D + lane * PER;
-      double acc = 0.0;
+    const bf16* xr = X + ((size_t)h * N + row) * D;
+    double best = DBL_MAX;
+    int bc = INT_MAX;
+    if (n > 0) {
+      float xv[PER];
 #pragma unroll
-      for (int t = 0; t < PER; ++t) {
-        const double df = (double)xv[t] - (double)mu[t];
-        acc = fma(df, df, acc);
+      for (int t = 0; t < PER; ++t) xv[t] = __bfloat162float(xr[lane * PER + t]);
+      for (int i = 0; i < n; ++i) {
+        const int c = e[3 + i];
+        const float* mu = cent + ((size_t)h * C + c) * D + lane * PER;
+        double acc = 0.0;
+#pragma unroll
+        for (int t = 0; t < PER; ++t) {
+          const double df = (double)xv[t] - (double)mu[t];
+          acc = fma(df, df, acc);
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+        if (acc < best || (acc == best && c < bc)) { best = acc; bc = c; }
+      }
+    } else {
+      for (int t = lane; t < D; t += 32) xs[wib][t] = __bfloat162float(xr[t]);
+      __syncwarp();
+      for (int c = lane; c < C; c += 32) {
+        const float4* mu = reinterpret_cast<const float4*>(cent + ((size_t)h * C + c) * D);
+        double acc = 0.0;
+#pragma unroll 8
+        for (int t4 = 0; t4 < D / 4; ++t4) {
+          const float4 m = mu[t4];
+          const double d0 = (double)xs[wib][4 * t4] - m.x, d1 = (double)xs[wib][4 * t4 + 1] - m.y;
+          const double d2 = (double)xs[wib][4 * t4 + 2] - m.z, d3 = (double)xs[wib][4 * t4 + 3] - m.w;
+          acc = fma(d0, d0, acc); acc = fma(d1, d1, acc); acc = fma(d2, d2, acc); acc = fma(d3, d3, acc);
+        }
+        if (acc < best || (acc == best && c < bc)) { best = acc; bc = c; }
       }
 #pragma unroll
-      for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
-      if (acc < best || (acc == best && c < bc)) { best = acc; bc = c; }
+      for (int o = 16; o > 0; o >>= 1) {
+        const double ob = __shfl_xor_sync(0xffffffffu, best, o);
+        const int oc = __shfl_xor_sync(0xffffffffu, bc, o);
+        if (ob < best || (ob == best && oc < bc)) { best = ob; bc = oc; }
+      }
+      __syncwarp();
     }
     if (lane == 0) labels[(size_t)h * N + row] = bc;
   }
 }
 
-template <int D>
-struct Smem {
-  static constexpr int kXBytes = BM * D * 2;
-  // offsets within the 1024-aligned dynamic shared memory
-  __host__ __device__ static int cent_off() { return 0; }
-  __host__ __device__ static int x_off(int Cpad) { return (Cpad * D * 2 + 1023) & ~1023; }
-  __host__ __device__ static int cn_off(int Cpad) { return x_off(Cpad) + 2 * kXBytes; }
-  __host__ __device__ static int merge_off(int Cpad) { return cn_off(Cpad) + ((Cpad * 4 + 15) & ~15); }
-  __host__ __device__ static int list_off(int Cpad) { return merge_off(Cpad) + BM * 4 * 4; }
-  __host__ __device__ static int bar_off(int Cpad) { return list_off(Cpad) + 2 * KC * 256 * 4; }
-  // at least 120 KB so that only one block (and one 512-column tensor-memory
-  // allocation) lives on an SM
-  static int total(int Cpad) { return std::max(bar_off(Cpad) + 16 * 8 + 1024, 120 * 1024); }
-};
+// Bound on |packed score - exact score| for a token of norm xn (see header):
+// xn ||mu - bf16(mu)|| for the centroid rounding, 2^-14 xn ||bf16(mu)|| for the
+// fp32 accumulation inside the MMA, a generous 2^-21 (||mu||^2 + 2 xn ||mu||)
+// for the rounding of ||mu||^2/2 and of the subtraction, and 2^(bits-23) |s|
+// for the index bits written over the mantissa.
+__device__ __forceinline__ float score_error(float xn, const Bounds& b, float idx_rel) {
+  const float mag = xn * b.mmax + 0.5f * b.nmax;
+  return xn * (b.dmax + 6.1035156e-5f * b.mmax) + 4.7683716e-7f * (b.nmax + 2.f * xn * b.mmax) +
+         idx_rel * mag * 1.0001f + 1e-30f;
+}
+
+// Insert two packed scores into the running top three (b1 >= b2 >= b3): the
+// k-th largest of two sorted lists is the largest min(A_i, B_j) over i + j = k.
+__device__ __forceinline__ void top3_add2(float& b1, float& b2, float& b3, float p0, float p1) {
+  const float hi = fmaxf(p0, p1), lo = fminf(p0, p1);
+  const float n3 = tc::fmax3(b3, fminf(b2, hi), fminf(b1, lo));
+  const float n2 = tc::fmax3(b2, fminf(b1, hi), lo);
+  b1 = fmaxf(b1, hi);
+  b2 = n2;
+  b3 = n3;
+}
+
+template <int NV>
+__device__ __forceinline__ void consume(const uint32_t (&v)[NV], const int4* __restrict__ tp, uint32_t keep,
+                                        float& b1, float& b2, float& b3) {
+#pragma unroll
+  for (int q = 0; q < NV; q += 2) {
+    const int4 e = tp[q >> 1];  // {||mu||^2/2, index} of two columns
+    const float s0 = __uint_as_float(v[q]) - __int_as_float(e.x);
+    const float s1 = __uint_as_float(v[q + 1]) - __int_as_float(e.z);
+    const float p0 = __uint_as_float((__float_as_uint(s0) & keep) | (uint32_t)e.y);
+    const float p1 = __uint_as_float((__float_as_uint(s1) & keep) | (uint32_t)e.w);
+    top3_add2(b1, b2, b3, p0, p1);
+  }
+}
 
 template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
-    k_assign_tc(const bf16* __restrict__ X, const bf16* __restrict__ cb, const float* __restrict__ cnorm,
-                const Bounds* __restrict__ bounds, const float* __restrict__ xnorm,
-                const float* __restrict__ cent, int N, int C, int Cpad, int tiles_per_cta,
-                int32_t* __restrict__ labels, int* __restrict__ refine, int* __restrict__ refine_count,
-                int* status) {
+    k_assign_tc(const __grid_constant__ CUtensorMap tmx, const __grid_constant__ CUtensorMap tmc,
+                const int2* __restrict__ table, const Bounds* __restrict__ bounds,
+                const float* __restrict__ xnorm, int N, int Cpad, int Cr, int stages, int tiles_per_cta,
+                int nbits, int32_t* __restrict__ labels, int* __restrict__ refine,
+                int* __restrict__ refine_count, int* status) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  using S = Smem<D>;
-  uint8_t* cent_s = smem + S::cent_off();
-  uint8_t* x_s = smem + S::x_off(Cpad);
-  float* cn_s = reinterpret_cast<float*>(smem + S::cn_off(Cpad));
-  int* merge = reinterpret_cast<int*>(smem + S::merge_off(Cpad));
-  float* list_s = reinterpret_cast<float*>(smem + S::list_off(Cpad));
-  int* list_c = reinterpret_cast<int*>(smem + S::list_off(Cpad) + KC * 256 * 4);
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + S::bar_off(Cpad));
-  uint64_t* cent_full = bars + 0;
-  uint64_t* x_full = bars + 1;     // [2]
-  uint64_t* x_empty = bars + 3;    // [2]
-  uint64_t* acc_full = bars + 5;   // [2]
-  uint64_t* acc_empty = bars + 7;  // [2]
-  uint64_t* done = bars + 9;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 10);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 11);
+  const Lay L = layout(D, Cr, Cpad, stages);
+  uint8_t* cent_s = smem + L.cent;
+  uint8_t* x_s = smem + L.x;
+  int2* tab = reinterpret_cast<int2*>(smem + L.tab);
+  float* mbuf = reinterpret_cast<float*>(smem + L.merge);  // [2][3][BM]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L.bars);
+  uint64_t* cent_full = bars;
+  uint64_t* x_full = bars + 1;                  // [kMaxStages]
+  uint64_t* x_empty = bars + 1 + kMaxStages;    // [kMaxStages]
+  uint64_t* acc_full = bars + 13;               // [kSlots]
+  uint64_t* acc_empty = bars + 17;              // [kSlots]
+  uint64_t* merge_full = bars + 21;             // [2]
+  uint64_t* merge_empty = bars + 23;            // [2]
+  uint64_t* done = bars + 25;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 26);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 27);
+  constexpr int kXBytes = BM * D * 2;
 
   const int h = blockIdx.y;
   const int T = (N + BM - 1) / BM;
   const int t0 = blockIdx.x * tiles_per_cta;
   const int nt = min(tiles_per_cta, T - t0);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int nchunk = (Cpad + kSlotCols - 1) / kSlotCols;
-  constexpr int CPR = D / 8;  // 16-byte chunks per row
+  const int nch = (Cpad + kChunk - 1) / kChunk;
 
   if (threadIdx.x == 0) {
-    tc::mbar_init(cent_full, kProducers);
-    for (int i = 0; i < 2; ++i) {
-      tc::mbar_init(x_full + i, kProducers);
+    tc::mbar_init(cent_full, 1);
+    for (int i = 0; i < stages; ++i) {
+      tc::mbar_init(x_full + i, 1);
       tc::mbar_init(x_empty + i, 1);
+    }
+    for (int i = 0; i < kSlots; ++i) {
       tc::mbar_init(acc_full + i, 1);
-      tc::mbar_init(acc_empty + i, 128);
+      tc::mbar_init(acc_empty + i, 4);
+    }
+    for (int i = 0; i < 2; ++i) {
+      tc::mbar_init(merge_full + i, 4);
+      tc::mbar_init(merge_empty + i, 4);
     }
     tc::mbar_init(done, 1);
     *abort_flag = 0;
     tc::mbar_fence_init();
   }
-  for (int c = threadIdx.x; c < Cpad; c += blockDim.x) cn_s[c] = cnorm[(size_t)h * Cpad + c];
+  for (int c = threadIdx.x; c < Cpad; c += blockDim.x) tab[c] = table[(size_t)h * Cpad + c];
   if (warp == 0) {
     tc::tmem_alloc(tmem_slot, 512);
     tc::tmem_relinquish();
@@ -278,164 +311,152 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) {
       bool ok = tc::mbar_wait(cent_full, 0, abort_flag, status);
       const uint32_t cent_a = tc::smem_u32(cent_s);
-      const uint32_t cregion = (uint32_t)Cpad * 128u;
+      const uint32_t cregion = (uint32_t)Cr * 128u;
+      int g = 0;
       for (int t = 0; ok && t < nt; ++t) {
-        const int stage = t & 1;
-        ok = tc::mbar_wait(x_full + stage, (t >> 1) & 1, abort_flag, status);
+        const int s = t % stages, k = t / stages;
+        ok = tc::mbar_wait(x_full + s, k & 1, abort_flag, status);
         if (!ok) break;
         tc::tc_fence_after();
-        const uint32_t xa = tc::smem_u32(x_s + stage * S::kXBytes);
-        for (int j = 0; j < nchunk; ++j) {
-          const int g = t * nchunk + j, slot = g & 1, use = g >> 1;
+        const uint32_t xa = tc::smem_u32(x_s + s * kXBytes);
+        for (int j = 0; j < nch; ++j, ++g) {
+          const int slot = g & (kSlots - 1), use = g >> 2;
           ok = tc::mbar_wait(acc_empty + slot, (use & 1) ^ 1, abort_flag, status);
           if (!ok) break;
           tc::tc_fence_after();
-          const int n0 = j * kSlotCols, nj = min(kSlotCols, Cpad - n0);
+          const int n0 = j * kChunk, nj = min(kChunk, Cpad - n0);
           const uint32_t id = tc::idesc_bf16(BM, nj, false, false);
-          for (int k = 0; k < D / 16; ++k) {
-            const uint64_t a = tc::desc_kmajor(xa, BM * 128u, k);
-            const uint64_t b = tc::desc_kmajor(cent_a + (uint32_t)n0 * 128u, cregion, k);
-            tc::mma_ss(tmem + (uint32_t)(slot * kSlotCols), a, b, id, k > 0 ? 1u : 0u);
+#pragma unroll
+          for (int k16 = 0; k16 < D / 16; ++k16) {
+            const uint64_t a = tc::desc_kmajor(xa, BM * 128u, k16);
+            const uint64_t b = tc::desc_kmajor(cent_a + (uint32_t)n0 * 128u, cregion, k16);
+            tc::mma_ss(tmem + (uint32_t)(slot * kChunk), a, b, id, k16 > 0 ? 1u : 0u);
           }
           tc::mma_commit(acc_full + slot);
         }
-        tc::mma_commit(x_empty + stage);
+        if (!ok) break;
+        tc::mma_commit(x_empty + s);
       }
       tc::mma_commit(done);
     }
     __syncwarp();
-  } else if (warp < 4) {
-    // ----------------------------------------------------------- producers
-    const int pt = threadIdx.x - 32;
-    const uint32_t cent_a = tc::smem_u32(cent_s);
-    const bf16* cbh = cb + (size_t)h * Cpad * D;
-    for (int e = pt; e < Cpad * CPR; e += kProducers) {
-      const int r = e / CPR, c = e % CPR;
-      tc::cp_async16(cent_a + tc::sw128_offset(r, c, Cpad), cbh + (size_t)r * D + c * 8, 16);
-    }
-    tc::cp_async_wait_all();
-    tc::fence_proxy_async();
-    tc::mbar_arrive(cent_full);
-    const bf16* Xh = X + (size_t)h * N * D;
-    for (int t = 0; t < nt; ++t) {
-      const int stage = t & 1;
-      if (!tc::mbar_wait(x_empty + stage, ((t >> 1) & 1) ^ 1, abort_flag, status)) break;
-      const uint32_t xa = tc::smem_u32(x_s + stage * S::kXBytes);
-      const int row0 = (t0 + t) * BM;
-      for (int e = pt; e < BM * CPR; e += kProducers) {
-        const int r = e / CPR, c = e % CPR;
-        const bool valid = row0 + r < N;
-        const bf16* src = Xh + (size_t)(valid ? row0 + r : 0) * D + c * 8;
-        tc::cp_async16(xa + tc::sw128_offset(r, c, BM), src, valid ? 16u : 0u);
+  } else if (warp == 1) {
+    // --------------------------------------------------------- TMA producer
+    if (lane == 0) {
+      tc::tma_prefetch_map(&tmx);
+      tc::tma_prefetch_map(&tmc);
+      const uint32_t cent_a = tc::smem_u32(cent_s);
+      tc::mbar_arrive_expect_tx(cent_full, (uint32_t)(Cr * D * 2));
+      for (int kh = 0; kh < D / 64; ++kh)
+        for (int rb = 0; rb < Cr / 128; ++rb)
+          tc::tma_load_3d(cent_a + (uint32_t)(kh * Cr * 128 + rb * 128 * 128), &tmc, kh * 64, rb * 128, h,
+                          cent_full);
+      for (int t = 0; t < nt; ++t) {
+        const int s = t % stages, k = t / stages;
+        if (!tc::mbar_wait(x_empty + s, (k & 1) ^ 1, abort_flag, status)) break;
+        const uint32_t xa = tc::smem_u32(x_s + s * kXBytes);
+        tc::mbar_arrive_expect_tx(x_full + s, (uint32_t)kXBytes);
+        for (int kh = 0; kh < D / 64; ++kh)
+          tc::tma_load_3d(xa + (uint32_t)(kh * BM * 128), &tmx, kh * 64, (t0 + t) * BM, h, x_full + s);
       }
-      tc::cp_async_wait_all();
-      tc::fence_proxy_async();
-      tc::mbar_arrive(x_full + stage);
     }
-    tc::cp_async_wait_all();
+    __syncwarp();
   } else {
     // ------------------------------------------------------------ epilogue
-    const int wg = (warp - 4) >> 2;           // 0 or 1
-    const int r = ((warp & 3) << 5) + lane;   // TMEM lane == tile row
+    const int wg = (warp - 2) >> 2;           // 0 or 1: takes chunks g with g % 2 == wg
+    const int quarter = warp & 3;             // TMEM lanes 32*quarter .. +31
+    const int r = quarter * 32 + lane;        // tile row == TMEM lane
+    const uint32_t keep = ~((1u << nbits) - 1u);
+    const float idx_rel = ldexpf(1.f, nbits - 23);
     const Bounds bd = bounds[h];
-    for (int t = 0; t < nt; ++t) {
-      const int row = (t0 + t) * BM + r;
-      const float xn = row < N ? xnorm[(size_t)h * N + row] : 0.f;
-      const float B = 2.f * xn * (bd.dmax + 6.1035e-5f * bd.mmax) +
-                      9.5367e-7f * (bd.nmax + 2.f * xn * bd.mmax) + 1e-30f;
-      const float W = 2.f * B;
-      const int et = threadIdx.x - 128;  // epilogue thread 0..255
-      float* ls = list_s + et;
-      int* lc = list_c + et;
-      Cands st{INFINITY, 0, 0};
+    bool ok = true;
+    for (int t = 0; t < nt && ok; ++t) {
+      float b1 = -INFINITY, b2 = -INFINITY, b3 = -INFINITY;
       bool mine = false;
-      for (int j = 0; j < nchunk; ++j) {
-        const int g = t * nchunk + j, slot = g & 1, use = g >> 1;
-        if (slot != wg) continue;
+      for (int j = 0; j < nch; ++j) {
+        const int g = t * nch + j;
+        if ((g & 1) != wg) continue;
         mine = true;
-        if (!tc::mbar_wait_warp(acc_full + slot, use & 1, abort_flag, status)) break;
+        const int slot = g & (kSlots - 1), use = g >> 2;
+        ok = tc::mbar_wait_warp(acc_full + slot, use & 1, abort_flag, status);
+        if (!ok) break;
         tc::tc_fence_after();
-        const int n0 = j * kSlotCols, nj = min(kSlotCols, Cpad - n0);
-        const uint32_t base = tc::taddr(tmem, (uint32_t)((warp & 3) << 5), (uint32_t)(slot * kSlotCols));
-        const int n32 = nj & ~31;
-        // pass 1: chunk minimum (padding columns score +inf)
-        float m = INFINITY;
-        for (int c0 = 0; c0 < n32; c0 += 32) {
-          uint32_t v[32];
-          tc::tmem_ld32(base + (uint32_t)c0, v);
+        const uint32_t base = tc::taddr(tmem, (uint32_t)(quarter * 32), (uint32_t)(slot * kChunk));
+        const int n0 = j * kChunk, nj = min(kChunk, Cpad - n0);
+        const int4* tp = reinterpret_cast<const int4*>(tab + n0);
+        int c0 = 0;
+        for (; c0 + 64 <= nj; c0 += 64) {
+          uint32_t va[32], vb[32];
+          tc::tmem_ld32(base + (uint32_t)c0, va);
+          tc::tmem_ld32(base + (uint32_t)(c0 + 32), vb);
           tc::tmem_ld_wait();
-          m = fminf(m, min32(v, cn_s + n0 + c0));
+          consume<32>(va, tp + (c0 >> 1), keep, b1, b2, b3);
+          consume<32>(vb, tp + ((c0 + 32) >> 1), keep, b1, b2, b3);
         }
-        if (n32 < nj) {
-          uint32_t v[16];
-          tc::tmem_ld16(base + (uint32_t)n32, v);
+        if (c0 + 32 <= nj) {
+          uint32_t va[32];
+          tc::tmem_ld32(base + (uint32_t)c0, va);
           tc::tmem_ld_wait();
-#pragma unroll
-          for (int q = 0; q < 16; ++q) m = fminf(m, fmaf(-2.f, __uint_as_float(v[q]), cn_s[n0 + n32 + q]));
+          consume<32>(va, tp + (c0 >> 1), keep, b1, b2, b3);
+          c0 += 32;
         }
-        if (m < st.best) {
-          st.best = m;
-          if (st.n) cand_compact(st, W, ls, lc);
-        }
-        // pass 2: every column within the window of the running minimum
-        const float thr = st.best + W;
-        for (int c0 = 0; c0 < n32; c0 += 32) {
-          uint32_t v[32];
-          tc::tmem_ld32(base + (uint32_t)c0, v);
+        if (c0 < nj) {  // nj is a multiple of 16
+          uint32_t va[16];
+          tc::tmem_ld16(base + (uint32_t)c0, va);
           tc::tmem_ld_wait();
-          collect<32>(st, v, cn_s + n0 + c0, n0 + c0, C, thr, ls, lc);
-        }
-        if (n32 < nj) {
-          uint32_t v[16];
-          tc::tmem_ld16(base + (uint32_t)n32, v);
-          tc::tmem_ld_wait();
-          collect<16>(st, v, cn_s + n0 + n32, n0 + n32, C, thr, ls, lc);
+          consume<16>(va, tp + (c0 >> 1), keep, b1, b2, b3);
         }
         tc::tc_fence_before();
-        tc::mbar_arrive(acc_empty + slot);
+        __syncwarp();
+        if (lane == 0) tc::mbar_arrive(acc_empty + slot);
       }
-      // on abort keep walking the tiles (waits now return at once) so that
-      // both warpgroups pass the same named barriers
-      bool finalize = mine;
-      if (nchunk >= 2) {
-        int* mrow = merge + r * 4;
-        if (wg == 1) { mrow[0] = __float_as_int(st.best); mrow[2] = st.n; mrow[3] = st.over; }
-        asm volatile("bar.sync 1, 256;" ::: "memory");
-        if (wg == 0) {
-          const float ob = __int_as_float(mrow[0]);
-          const int on = mrow[2];
-          st.over |= mrow[3];
-          if (ob < st.best) {
-            st.best = ob;
-            if (st.n) cand_compact(st, W, ls, lc);
-          }
-          const float thr = st.best + W;
-          for (int i = 0; i < min(on, KC); ++i) {
-            const float os = list_s[i * 256 + et + 128];
-            if (os <= thr) cand_push(st, os, list_c[i * 256 + et + 128], ls, lc);
-          }
-          if (on > KC) st.over = 1;
+      if (!ok || !mine) continue;
+      // the tile's last chunk decides; the other warpgroup (if it had chunks
+      // of this tile) hands over its partial top three
+      const bool decider = ((t * nch + nch - 1) & 1) == wg;
+      const int mb = t & 1;
+      const uint32_t mpar = (uint32_t)(t >> 1) & 1u;
+      float* mrow = mbuf + mb * 3 * BM + r;
+      if (nch >= 2 && !decider) {
+        ok = tc::mbar_wait_warp(merge_empty + mb, mpar ^ 1u, abort_flag, status);
+        if (!ok) break;
+        mrow[0] = b1; mrow[BM] = b2; mrow[2 * BM] = b3;
+        __syncwarp();
+        if (lane == 0) tc::mbar_arrive(merge_full + mb);
+        continue;
+      }
+      if (nch >= 2) {
+        ok = tc::mbar_wait_warp(merge_full + mb, mpar, abort_flag, status);
+        if (!ok) break;
+        const float c1 = mrow[0], c2 = mrow[BM], c3 = mrow[2 * BM];
+        __syncwarp();
+        if (lane == 0) tc::mbar_arrive(merge_empty + mb);
+        const float n3 = fmaxf(tc::fmax3(b3, fminf(b2, c1), fminf(b1, c2)), c3);
+        const float n2 = tc::fmax3(b2, fminf(b1, c1), c2);
+        b1 = fmaxf(b1, c1);
+        b2 = n2;
+        b3 = n3;
+      }
+      const int row = (t0 + t) * BM + r;
+      int need = 0, lab = 0;
+      if (row < N) {
+        const float xn = xnorm[(size_t)h * N + row];
+        const float thr = b1 - 2.02f * score_error(xn, bd, idx_rel);
+        lab = (int)(__float_as_uint(b1) & ~keep);
+        need = b2 >= thr ? (b3 >= thr ? -1 : 2) : 0;
+        labels[(size_t)h * N + row] = lab;
+      }
+      // several centroids within the bound: listed for the float64 pass
+      const uint32_t want = __ballot_sync(0xffffffffu, need != 0);
+      if (want) {
+        int base = 0;
+        if (lane == 0) base = atomicAdd(refine_count, __popc(want));
+        base = __shfl_sync(0xffffffffu, base, 0);
+        if (need) {
+          int* e = refine + (size_t)(base + __popc(want & ((1u << lane) - 1u))) * kRefineInts;
+          e[0] = h; e[1] = row; e[2] = need; e[3] = lab;
+          e[4] = (int)(__float_as_uint(b2) & ~keep);
         }
-        asm volatile("bar.sync 1, 256;" ::: "memory");
-        finalize = wg == 0;
-      }
-      if (!finalize || row >= N || *abort_flag) continue;
-      // the listed candidate with the smallest score (smaller index on ties)
-      cand_compact(st, W, ls, lc);
-      int label = 0;
-      float bs = INFINITY;
-      for (int i = 0; i < min(st.n, KC); ++i) {
-        const float v = ls[i * 256];
-        const int c = lc[i * 256];
-        if (v < bs || (v == bs && c < label)) { bs = v; label = c; }
-      }
-      labels[(size_t)h * N + row] = label;
-      if (st.n > 1 || st.over) {
-        // several centroids within the bound: decided later in float64
-        const int k = atomicAdd(refine_count, 1);
-        int* e = refine + (size_t)k * kRefineInts;
-        e[0] = h; e[1] = row; e[2] = st.over ? -1 : st.n;
-        for (int i = 0; i < min(st.n, KC); ++i) e[3 + i] = lc[i * 256];
       }
     }
   }
@@ -452,33 +473,46 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 }  // namespace
 
+static int pick_stages(int d, int C) {
+  const int Cpad = round16(C), Cr = round128(C);
+  int s = 0;
+  while (s < kMaxStages && layout(d, Cr, Cpad, s + 1).total <= kSmemLimit) ++s;
+  return s;
+}
+
 bool kmeans_tc_supported(int d, int C) {
   if (d != 64 && d != 128) return false;
-  return round16(C) * d * 2 <= kCentBytesMax;
+  if (C < 1 || C > kMaxC) return false;
+  return pick_stages(d, C) >= 2;
+}
+
+bool kmeans_tc_usable(const void* X, int N, int d, int C) {
+  return kmeans_tc_supported(d, C) && N >= BM && (reinterpret_cast<uintptr_t>(X) & 15u) == 0 &&
+         tma_available();
 }
 
 // Workspace: token norms [H,N] first (they only depend on H, N), then the
-// per-iteration centroid copy, norms and bounds, and the list of rows left
-// for the float64 pass with its counter.
+// per-pass centroid copy and table, the bounds with the refine counter right
+// behind them (cleared together), and the list of rows for the float64 pass.
 struct TcWs {
   float* xn;
   bf16* cb;
-  float* cn;
+  int2* table;
   Bounds* bd;
-  int* refine;
   int* refine_count;
+  int* refine;
 };
 
 static size_t tc_layout(int H, int N, int d, int C, TcWs* out, void* ws) {
   Carve cv(ws);
-  const int Cpad = round16(C);
+  const int Cpad = round16(C), Cr = round128(C);
   TcWs w;
   w.xn = cv.take<float>((size_t)H * N);
-  w.cb = cv.take<bf16>((size_t)H * Cpad * d);
-  w.cn = cv.take<float>((size_t)H * Cpad);
-  w.bd = cv.take<Bounds>(H);
+  w.cb = cv.take<bf16>((size_t)H * Cr * d);
+  w.table = cv.take<int2>((size_t)H * Cpad);
+  w.bd = cv.take<Bounds>((size_t)H + 1);
+  w.refine_count = reinterpret_cast<int*>(w.bd ? w.bd + H : nullptr);
   w.refine = cv.take<int>((size_t)H * N * kRefineInts);
-  w.refine_count = cv.take<int>(1);
   if (out) *out = w;
   return cv.used();
 }
@@ -492,8 +526,49 @@ cudaError_t kmeans_tc_prepare_rows(const void* Xv, int H, int N, int d, void* ws
   float* xn = static_cast<float*>(ws);  // first buffer of the layout above
   const bf16* X = static_cast<const bf16*>(Xv);
   const long long rows = (long long)H * N;
-  if (d == 128) { k_row_norms<128><<<(unsigned)((rows + 7) / 8), 256, 0, st>>>(X, rows, xn); note_launch(); }
-  else { k_row_norms<64><<<(unsigned)((rows + 7) / 8), 256, 0, st>>>(X, rows, xn); note_launch(); }
+  const int rpb = 8 * (256 / d);  // rows per block and pass: 8 warps x 32/(d/8)
+  const unsigned grid = (unsigned)std::min<long long>((rows + rpb - 1) / rpb, 148LL * 16);
+  if (d == 128) { k_row_norms<128><<<grid, 256, 0, st>>>(X, rows, xn); note_launch(); }
+  else { k_row_norms<64><<<grid, 256, 0, st>>>(X, rows, xn); note_launch(); }
+  return cudaGetLastError();
+}
+
+// Tiles per block: the count that minimises (waves of 148 blocks) x (tiles per
+// block + a setup cost of about three tiles).
+static int pick_tiles_per_cta(int H, int T) {
+  int best = 1;
+  long long best_cost = LLONG_MAX;
+  for (int tpc = 4; tpc <= 64; ++tpc) {
+    const long long ctas = (long long)H * ((T + tpc - 1) / tpc);
+    const long long cost = ((ctas + 147) / 148) * (tpc + 3);
+    if (cost < best_cost) { best_cost = cost; best = tpc; }
+  }
+  return std::min(best, std::max(1, T));
+}
+
+template <int D>
+static cudaError_t assign_launch(const bf16* X, int H, int N, int C, const float* cent, int32_t* labels,
+                                 const TcWs& w, cudaStream_t st) {
+  const int Cpad = round16(C), Cr = round128(C);
+  const int stages = pick_stages(D, C);
+  int nbits = 1;
+  while ((1 << nbits) < Cpad) ++nbits;
+  k_prep_centroids<D><<<dim3(Cr / 8, H), 256, 0, st>>>(cent, C, Cpad, Cr, w.cb, w.table, w.bd);
+  note_launch();
+  CUtensorMap tmx, tmc;
+  if (!tma_map_bf16_3d(&tmx, X, D, N, H, BM) || !tma_map_bf16_3d(&tmc, w.cb, D, Cr, H, 128))
+    return cudaErrorInvalidValue;
+  const int smem = layout(D, Cr, Cpad, stages).total;
+  cudaError_t e = cudaFuncSetAttribute(k_assign_tc<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return e;
+  const int T = (N + BM - 1) / BM;
+  const int tpc = pick_tiles_per_cta(H, T);
+  k_assign_tc<D><<<dim3((T + tpc - 1) / tpc, H), kThreads, smem, st>>>(
+      tmx, tmc, w.table, w.bd, w.xn, N, Cpad, Cr, stages, tpc, nbits, labels, w.refine, w.refine_count,
+      status_word());
+  note_launch();
+  k_refine<D><<<148 * 4, 256, 0, st>>>(X, cent, N, C, w.refine, w.refine_count, labels);
+  note_launch();
   return cudaGetLastError();
 }
 
@@ -501,33 +576,11 @@ cudaError_t kmeans_assign_tc(const void* Xv, int H, int N, int d, int C, const f
                              int32_t* labels, void* ws, cudaStream_t st) {
   TcWs w;
   tc_layout(H, N, d, C, &w, ws);
-  const int Cpad = round16(C);
-  const bf16* X = static_cast<const bf16*>(Xv);
-  const int T = (N + BM - 1) / BM;
-  const int tpc = std::max(1, std::min(16, (int)((long long)H * T / (2 * 148))));
-  const int gx = (T + tpc - 1) / tpc;
-  cudaError_t e = cudaMemsetAsync(w.refine_count, 0, sizeof(int), st);
+  cudaError_t e = cudaMemsetAsync(w.bd, 0, sizeof(Bounds) * ((size_t)H + 1), st);
   if (e != cudaSuccess) return e;
-  if (d == 128) {
-    k_prep_centroids<128><<<H, 256, 0, st>>>(cent, C, Cpad, w.cb, w.cn, w.bd); note_launch();
-    const int smem = Smem<128>::total(Cpad);
-    e = cudaFuncSetAttribute(k_assign_tc<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-    if (e != cudaSuccess) return e;
-    k_assign_tc<128><<<dim3(gx, H), kThreads, smem, st>>>(X, w.cb, w.cn, w.bd, w.xn, cent, N, C, Cpad, tpc,
-                                                           labels, w.refine, w.refine_count, status_word());
-    note_launch();
-    k_refine<128><<<148 * 8, 256, 0, st>>>(X, cent, N, C, w.refine, w.refine_count, labels); note_launch();
-  } else {
-    k_prep_centroids<64><<<H, 256, 0, st>>>(cent, C, Cpad, w.cb, w.cn, w.bd); note_launch();
-    const int smem = Smem<64>::total(Cpad);
-    e = cudaFuncSetAttribute(k_assign_tc<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-    if (e != cudaSuccess) return e;
-    k_assign_tc<64><<<dim3(gx, H), kThreads, smem, st>>>(X, w.cb, w.cn, w.bd, w.xn, cent, N, C, Cpad, tpc,
-                                                          labels, w.refine, w.refine_count, status_word());
-    note_launch();
-    k_refine<64><<<148 * 8, 256, 0, st>>>(X, cent, N, C, w.refine, w.refine_count, labels); note_launch();
-  }
-  return cudaGetLastError();
+  const bf16* X = static_cast<const bf16*>(Xv);
+  if (d == 128) return assign_launch<128>(X, H, N, C, cent, labels, w, st);
+  return assign_launch<64>(X, H, N, C, cent, labels, w, st);
 }
 
 }  // namespace svg

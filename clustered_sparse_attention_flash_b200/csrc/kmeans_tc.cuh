@@ -6,6 +6,9 @@
 
 namespace svg {
 bool kmeans_tc_supported(int d, int C);
+// Supported shape, at least one full tile of tokens, 16-byte aligned tokens
+// and a driver that encodes TMA maps.
+bool kmeans_tc_usable(const void* X, int N, int d, int C);
 size_t kmeans_tc_ws_bytes(int H, int N, int d, int C);
 // Once per k-means call: per-token norms used by the rounding bound.
 cudaError_t kmeans_tc_prepare_rows(const void* X, int H, int N, int d, void* ws, cudaStream_t st);

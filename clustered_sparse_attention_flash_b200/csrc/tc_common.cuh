@@ -273,6 +273,30 @@ __device__ __forceinline__ void cp_async_wait_group() {
   asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
 }
 
+// ---------------------------------------------------- TMA tensor copies
+
+// Tiled copy of one box of a 3-D tensor map (coordinates x innermost, in
+// elements) into shared memory, completing as transaction bytes on `bar`.
+// The map lives in kernel parameter space (a __grid_constant__ argument).
+__device__ __forceinline__ void tma_load_3d(uint32_t dst, const void* map, int x, int y, int z,
+                                            uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes "
+      "[%0], [%1, {%2, %3, %4}], [%5];" ::"r"(dst),
+      "l"(map), "r"(x), "r"(y), "r"(z), "r"(smem_u32(bar))
+      : "memory");
+}
+__device__ __forceinline__ void tma_prefetch_map(const void* map) {
+  asm volatile("prefetch.tensormap [%0];" ::"l"(map) : "memory");
+}
+
+// Three-input float maximum (one instruction on sm_100).
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+
 // Byte offset of 16-byte chunk `c` (of a bf16 row with D/8 chunks) of row `r`
 // inside an SW128 K-major tile of `rows` rows.
 __device__ __forceinline__ uint32_t sw128_offset(int r, int c, int rows) {
