@@ -80,12 +80,12 @@ __global__ void __launch_bounds__(256) k_update(const T* __restrict__ X, const i
 #pragma unroll
   for (int t = 0; t < PER; ++t) acc[t] = 0.0;
   int r = beg + w;
-  for (; r + 3 * NW < end; r += 4 * NW) {
-    int idx[4];
+  for (; r + 7 * NW < end; r += 8 * NW) {
+    int idx[8];
 #pragma unroll
-    for (int u = 0; u < 4; ++u) idx[u] = ph[r + u * NW];
+    for (int u = 0; u < 8; ++u) idx[u] = ph[r + u * NW];
 #pragma unroll
-    for (int u = 0; u < 4; ++u) {
+    for (int u = 0; u < 8; ++u) {
       if constexpr (PER == 4) {
         float4 v = ld4(Xh + (size_t)idx[u] * D);
         acc[0] += v.x; acc[1] += v.y; acc[2] += v.z; acc[3] += v.w;

@@ -43,7 +43,6 @@ constexpr int kThreads = 320;
 constexpr int kChunk = 128;            // accumulator columns per TMEM slot
 constexpr int kSlots = 4;
 constexpr int kMaxStages = 6;
-constexpr int kRefineInts = 8;         // h, row, n (2, or -1 = all centroids), c1, c2, pad
 constexpr int kSmemLimit = 232448;     // opt-in dynamic shared memory per block
 constexpr int kMaxC = 1024;            // index bits packed into the score: at most 10
 constexpr float kPadHalfNorm = 1e30f;  // ||mu||^2/2 of padding columns: never best, finite
@@ -73,21 +72,30 @@ __host__ __device__ inline Lay layout(int D, int Cr, int Cpad, int stages) {
   return l;
 }
 
-// Per centroid row (one warp each): bf16 copy (zero rows up to Cr), the table
-// entry {||mu||^2 / 2, index} (padding columns up to Cpad get kPadHalfNorm) and
+// Per block of 32 centroid rows of one head: the bf16 copy (zero rows up to
+// Cr), the table entry {||mu||^2 / 2, index} (padding columns up to Cpad get
+// kPadHalfNorm), a transposed float32 copy [d][C] for the float64 pass, and
 // the per-head maxima of the error bound.
 template <int D>
 __global__ void __launch_bounds__(256) k_prep_centroids(const float* __restrict__ cent, int C, int Cpad, int Cr,
                                                         bf16* __restrict__ cb, int2* __restrict__ table,
-                                                        Bounds* __restrict__ bounds) {
+                                                        float* __restrict__ centT, Bounds* __restrict__ bounds) {
+  __shared__ float tile[32][D + 1];
   __shared__ float red[3][8];
-  const int h = blockIdx.y, w = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int c = blockIdx.x * 8 + w;
+  const int h = blockIdx.y, c0 = blockIdx.x * 32;
+  const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  for (int e = threadIdx.x; e < 32 * D; e += blockDim.x) {
+    const int r = e / D, t = e % D, c = c0 + r;
+    tile[r][t] = c < C ? cent[((size_t)h * C + c) * D + t] : 0.f;
+  }
+  __syncthreads();
   float dmax = 0.f, mmax = 0.f, nmax = 0.f;
-  if (c < Cr) {
+  for (int r = w; r < 32; r += 8) {
+    const int c = c0 + r;
+    if (c >= Cr) break;
     double dn = 0.0, mb = 0.0, n2 = 0.0;
     for (int t = lane; t < D; t += 32) {
-      const float m = c < C ? cent[((size_t)h * C + c) * D + t] : 0.f;
+      const float m = tile[r][t];
       const bf16 b = __float2bfloat16_rn(m);
       cb[((size_t)h * Cr + c) * D + t] = b;
       const double bd = (double)__bfloat162float(b);
@@ -103,10 +111,14 @@ __global__ void __launch_bounds__(256) k_prep_centroids(const float* __restrict_
     if (lane == 0 && c < Cpad)
       table[(size_t)h * Cpad + c] = make_int2(__float_as_int(c < C ? (float)(0.5 * n2) : kPadHalfNorm), c);
     if (c < C) {
-      dmax = (float)sqrt(dn);
-      mmax = (float)sqrt(mb);
-      nmax = (float)n2;
+      dmax = fmaxf(dmax, (float)sqrt(dn));
+      mmax = fmaxf(mmax, (float)sqrt(mb));
+      nmax = fmaxf(nmax, (float)n2);
     }
+  }
+  for (int e = threadIdx.x; e < 32 * D; e += blockDim.x) {
+    const int t = e / 32, r = e % 32, c = c0 + r;
+    if (c < C) centT[((size_t)h * D + t) * C + c] = tile[r][t];
   }
   if (lane == 0) { red[0][w] = dmax; red[1][w] = mmax; red[2][w] = nmax; }
   __syncthreads();
@@ -145,56 +157,183 @@ __global__ void __launch_bounds__(256) k_row_norms(const bf16* __restrict__ X, l
   }
 }
 
-// Rows the tensor-core pass left ambiguous, one warp each: float64 distances
-// ||x - mu_c||^2 to the two listed candidates (lanes split the dimensions), or
-// to every centroid (lanes split the centroids); the smallest wins, the
-// smaller index on ties.
+// Rows the tensor-core pass left with two candidates {c1, c2}: float64
+// distances ||x - mu_c||^2 to both, the smaller wins (the smaller index on
+// ties).  Eight lanes per row, four rows per warp.
 template <int D>
-__global__ void __launch_bounds__(256) k_refine(const bf16* __restrict__ X, const float* __restrict__ cent,
-                                                int N, int C, const int* __restrict__ refine,
-                                                const int* __restrict__ count, int32_t* __restrict__ labels) {
-  constexpr int PER = D / 32;
-  __shared__ float xs[8][D];
-  const int lane = threadIdx.x & 31, wib = threadIdx.x >> 5;
-  const int nw = gridDim.x * (blockDim.x >> 5);
+__global__ void __launch_bounds__(256) k_refine2(const bf16* __restrict__ X, const float* __restrict__ cent,
+                                                 int N, int C, const int4* __restrict__ list,
+                                                 const int* __restrict__ count, int32_t* __restrict__ labels) {
+  constexpr int PER = D / 8;  // dimensions per lane
+  const int lane = threadIdx.x & 31, sub = lane & 7;
   const int total = *count;
-  for (int w = blockIdx.x * (blockDim.x >> 5) + wib; w < total; w += nw) {
-    const int* e = refine + (size_t)w * kRefineInts;
-    const int h = e[0], row = e[1], n = e[2];
-    const bf16* xr = X + ((size_t)h * N + row) * D;
-    double best = DBL_MAX;
-    int bc = INT_MAX;
-    if (n > 0) {
-      float xv[PER];
+  const int nwarps = gridDim.x * (blockDim.x >> 5);
+  for (int wb = (blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5)) * 4; wb < total; wb += nwarps * 4) {
+    const int gi = wb + (lane >> 3);
+    const bool act = gi < total;
+    int4 e = make_int4(0, 0, 0, 0);
+    if (act) e = list[gi];
+    double a0 = 0.0, a1 = 0.0;
+    if (act) {
+      const bf16* xr = X + ((size_t)e.x * N + e.y) * D + sub * PER;
+      const float* m0 = cent + ((size_t)e.x * C + e.z) * D + sub * PER;
+      const float* m1 = cent + ((size_t)e.x * C + e.w) * D + sub * PER;
 #pragma unroll
-      for (int t = 0; t < PER; ++t) xv[t] = __bfloat162float(xr[lane * PER + t]);
-      for (int i = 0; i < n; ++i) {
-        const int c = e[3 + i];
-        const float* mu = cent + ((size_t)h * C + c) * D + lane * PER;
-        double acc = 0.0;
+      for (int t = 0; t < PER; t += 4) {
+        const float2 xa = ld2(xr + t), xb = ld2(xr + t + 2);
+        const float4 u = *reinterpret_cast<const float4*>(m0 + t);
+        const float4 w = *reinterpret_cast<const float4*>(m1 + t);
+        const double x4[4] = {xa.x, xa.y, xb.x, xb.y};
+        const double u4[4] = {u.x, u.y, u.z, u.w}, w4[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
-        for (int t = 0; t < PER; ++t) {
-          const double df = (double)xv[t] - (double)mu[t];
-          acc = fma(df, df, acc);
+        for (int i = 0; i < 4; ++i) {
+          const double du = x4[i] - u4[i], dw = x4[i] - w4[i];
+          a0 = fma(du, du, a0);
+          a1 = fma(dw, dw, a1);
         }
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
-        if (acc < best || (acc == best && c < bc)) { best = acc; bc = c; }
       }
-    } else {
-      for (int t = lane; t < D; t += 32) xs[wib][t] = __bfloat162float(xr[t]);
-      __syncwarp();
-      for (int c = lane; c < C; c += 32) {
-        const float4* mu = reinterpret_cast<const float4*>(cent + ((size_t)h * C + c) * D);
-        double acc = 0.0;
-#pragma unroll 8
-        for (int t4 = 0; t4 < D / 4; ++t4) {
-          const float4 m = mu[t4];
-          const double d0 = (double)xs[wib][4 * t4] - m.x, d1 = (double)xs[wib][4 * t4 + 1] - m.y;
-          const double d2 = (double)xs[wib][4 * t4 + 2] - m.z, d3 = (double)xs[wib][4 * t4 + 3] - m.w;
-          acc = fma(d0, d0, acc); acc = fma(d1, d1, acc); acc = fma(d2, d2, acc); acc = fma(d3, d3, acc);
+    }
+#pragma unroll
+    for (int o = 4; o > 0; o >>= 1) {
+      a0 += __shfl_xor_sync(0xffffffffu, a0, o);
+      a1 += __shfl_xor_sync(0xffffffffu, a1, o);
+    }
+    if (act && sub == 0)
+      labels[(size_t)e.x * N + e.y] = (a1 < a0 || (a1 == a0 && e.w < e.z)) ? e.w : e.z;
+  }
+}
+
+// Rows with three or more candidates, listed per head: every centroid is
+// scanned in float32, eight rows at a time (a thread owns centroids tid,
+// tid + blockDim, ... and keeps the eight rows' distances, so each coalesced
+// load of the transposed centroids serves eight rows).  With d + 3 roundings
+// per distance the float32 value is within (d + 3) 2^-24 of the exact one in
+// relative terms, so every centroid whose float32 distance is within a
+// relative 2e-5 of the row's smallest is a candidate: a single candidate is
+// the nearest centroid, several (ties within the float32 error) are re-checked
+// in float64 by their threads; the smallest float64 distance wins, the
+// smaller index on ties.
+constexpr int kFullRows = 8;
+constexpr int kFullThreads = 256;
+
+template <int D>
+__global__ void __launch_bounds__(kFullThreads) k_refine_full(const bf16* __restrict__ X,
+                                                              const float* __restrict__ cent,
+                                                              const float* __restrict__ centT, int N, int C,
+                                                              const int* __restrict__ list,
+                                                              const int* __restrict__ counts,
+                                                              int32_t* __restrict__ labels) {
+  constexpr int R = kFullRows;
+  constexpr int KMAX = kMaxC / kFullThreads;  // centroids per thread: blocks of 256 when C > 256
+  __shared__ __align__(16) float xs[D][R];
+  __shared__ float rmin[R][kFullThreads / 32];
+  __shared__ double rbest[R][kFullThreads / 32];
+  __shared__ int rbc[R][kFullThreads / 32];
+  __shared__ int rcnt[R][kFullThreads / 32];
+  __shared__ int rtie[R];
+  const int h = blockIdx.y;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, nwarp = blockDim.x >> 5;
+  const int total = counts[h];
+  const int* lh = list + (size_t)h * N;
+  const float* cth = centT + (size_t)h * D * C;
+  const float* ch = cent + (size_t)h * C * D;
+  for (int base = blockIdx.x * R; base < total; base += gridDim.x * R) {
+    for (int e = tid; e < D * R; e += blockDim.x) {
+      const int r = e / D, t = e % D;
+      xs[t][r] = base + r < total ? __bfloat162float(X[((size_t)h * N + lh[base + r]) * D + t]) : 0.f;
+    }
+    __syncthreads();
+    float dl[KMAX][R];
+    float dmin[R];
+#pragma unroll
+    for (int r = 0; r < R; ++r) dmin[r] = INFINITY;
+#pragma unroll
+    for (int k = 0; k < KMAX; ++k) {
+      const int c = k * blockDim.x + tid;
+#pragma unroll
+      for (int r = 0; r < R; ++r) dl[k][r] = INFINITY;
+      if (k * (int)blockDim.x >= C) continue;
+      if (c < C) {
+        float acc[R];
+#pragma unroll
+        for (int r = 0; r < R; ++r) acc[r] = 0.f;
+#pragma unroll 16
+        for (int t = 0; t < D; ++t) {
+          const float m = cth[(size_t)t * C + c];
+          const float4 xa = *reinterpret_cast<const float4*>(&xs[t][0]);
+          const float4 xb = *reinterpret_cast<const float4*>(&xs[t][4]);
+          const float xv[R] = {xa.x, xa.y, xa.z, xa.w, xb.x, xb.y, xb.z, xb.w};
+#pragma unroll
+          for (int r = 0; r < R; ++r) {
+            const float df = xv[r] - m;
+            acc[r] = fmaf(df, df, acc[r]);
+          }
         }
-        if (acc < best || (acc == best && c < bc)) { best = acc; bc = c; }
+#pragma unroll
+        for (int r = 0; r < R; ++r) {
+          dl[k][r] = acc[r];
+          dmin[r] = fminf(dmin[r], acc[r]);
+        }
+      }
+    }
+#pragma unroll
+    for (int r = 0; r < R; ++r) {
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) dmin[r] = fminf(dmin[r], __shfl_xor_sync(0xffffffffu, dmin[r], o));
+      if (lane == 0) rmin[r][warp] = dmin[r];
+    }
+    __syncthreads();
+    // rows whose window holds a single centroid are decided; the others
+    // (ties within the float32 error) go through float64
+    float lim[R];
+#pragma unroll
+    for (int r = 0; r < R; ++r) {
+      float g = INFINITY;
+      for (int i = 0; i < nwarp; ++i) g = fminf(g, rmin[r][i]);
+      lim[r] = g * (1.f + 2e-5f) + 1e-30f;
+      int n = 0, cmin = INT_MAX;
+#pragma unroll
+      for (int k = 0; k < KMAX; ++k) {
+        const int c = k * blockDim.x + tid;
+        if (c < C && dl[k][r] <= lim[r]) { ++n; cmin = min(cmin, c); }
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+        n += __shfl_xor_sync(0xffffffffu, n, o);
+        cmin = min(cmin, __shfl_xor_sync(0xffffffffu, cmin, o));
+      }
+      if (lane == 0) { rcnt[r][warp] = n; rbc[r][warp] = cmin; }
+    }
+    __syncthreads();
+    if (tid < R) {
+      int n = 0, cmin = INT_MAX;
+      for (int i = 0; i < nwarp; ++i) { n += rcnt[tid][i]; cmin = min(cmin, rbc[tid][i]); }
+      rtie[tid] = n > 1;
+      if (base + tid < total && n == 1) labels[(size_t)h * N + lh[base + tid]] = cmin;
+    }
+    __syncthreads();
+#pragma unroll
+    for (int r = 0; r < R; ++r) {
+      if (!rtie[r] || base + r >= total) continue;  // block-uniform
+      double best = DBL_MAX;
+      int bc = INT_MAX;
+#pragma unroll
+      for (int k = 0; k < KMAX; ++k) {
+        const int c = k * blockDim.x + tid;
+        if (c < C && dl[k][r] <= lim[r]) {
+          const float4* mu = reinterpret_cast<const float4*>(ch + (size_t)c * D);
+          double a4[4] = {0.0, 0.0, 0.0, 0.0};
+#pragma unroll 4
+          for (int t4 = 0; t4 < D / 4; ++t4) {
+            const float4 m = mu[t4];
+            const double d0 = (double)xs[4 * t4][r] - m.x, d1 = (double)xs[4 * t4 + 1][r] - m.y;
+            const double d2 = (double)xs[4 * t4 + 2][r] - m.z, d3 = (double)xs[4 * t4 + 3][r] - m.w;
+            a4[0] = fma(d0, d0, a4[0]); a4[1] = fma(d1, d1, a4[1]);
+            a4[2] = fma(d2, d2, a4[2]); a4[3] = fma(d3, d3, a4[3]);
+          }
+          const double acc = (a4[0] + a4[1]) + (a4[2] + a4[3]);
+          if (acc < best || (acc == best && c < bc)) { best = acc; bc = c; }
+        }
       }
 #pragma unroll
       for (int o = 16; o > 0; o >>= 1) {
@@ -202,9 +341,20 @@ __global__ void __launch_bounds__(256) k_refine(const bf16* __restrict__ X, cons
         const int oc = __shfl_xor_sync(0xffffffffu, bc, o);
         if (ob < best || (ob == best && oc < bc)) { best = ob; bc = oc; }
       }
-      __syncwarp();
+      if (lane == 0) { rbest[r][warp] = best; rbc[r][warp] = bc; }
     }
-    if (lane == 0) labels[(size_t)h * N + row] = bc;
+    __syncthreads();
+    if (tid < R && rtie[tid] && base + tid < total) {
+      double bb = rbest[tid][0];
+      int cc = rbc[tid][0];
+      for (int i = 1; i < nwarp; ++i) {
+        const double ob = rbest[tid][i];
+        const int oc = rbc[tid][i];
+        if (ob < bb || (ob == bb && oc < cc)) { bb = ob; cc = oc; }
+      }
+      labels[(size_t)h * N + lh[base + tid]] = cc;
+    }
+    __syncthreads();
   }
 }
 
@@ -249,8 +399,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     k_assign_tc(const __grid_constant__ CUtensorMap tmx, const __grid_constant__ CUtensorMap tmc,
                 const int2* __restrict__ table, const Bounds* __restrict__ bounds,
                 const float* __restrict__ xnorm, int N, int Cpad, int Cr, int stages, int tiles_per_cta,
-                int nbits, int32_t* __restrict__ labels, int* __restrict__ refine,
-                int* __restrict__ refine_count, int* status) {
+                int nbits, int32_t* __restrict__ labels, int4* __restrict__ list2,
+                int* __restrict__ list_full, int* __restrict__ counts, int* status) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const Lay L = layout(D, Cr, Cpad, stages);
@@ -446,17 +596,23 @@ __global__ void __launch_bounds__(kThreads, 1)
         need = b2 >= thr ? (b3 >= thr ? -1 : 2) : 0;
         labels[(size_t)h * N + row] = lab;
       }
-      // several centroids within the bound: listed for the float64 pass
-      const uint32_t want = __ballot_sync(0xffffffffu, need != 0);
-      if (want) {
+      // several centroids within the bound: listed for the float64 passes
+      const uint32_t want2 = __ballot_sync(0xffffffffu, need == 2);
+      const uint32_t wantf = __ballot_sync(0xffffffffu, need < 0);
+      const uint32_t below = (1u << lane) - 1u;
+      if (want2) {
         int base = 0;
-        if (lane == 0) base = atomicAdd(refine_count, __popc(want));
+        if (lane == 0) base = atomicAdd(counts, __popc(want2));
         base = __shfl_sync(0xffffffffu, base, 0);
-        if (need) {
-          int* e = refine + (size_t)(base + __popc(want & ((1u << lane) - 1u))) * kRefineInts;
-          e[0] = h; e[1] = row; e[2] = need; e[3] = lab;
-          e[4] = (int)(__float_as_uint(b2) & ~keep);
-        }
+        if (need == 2)
+          list2[base + __popc(want2 & below)] =
+              make_int4(h, row, lab, (int)(__float_as_uint(b2) & ~keep));
+      }
+      if (wantf) {
+        int base = 0;
+        if (lane == 0) base = atomicAdd(counts + 1 + h, __popc(wantf));
+        base = __shfl_sync(0xffffffffu, base, 0);
+        if (need < 0) list_full[(size_t)h * N + base + __popc(wantf & below)] = row;
       }
     }
   }
@@ -492,16 +648,21 @@ bool kmeans_tc_usable(const void* X, int N, int d, int C) {
 }
 
 // Workspace: token norms [H,N] first (they only depend on H, N), then the
-// per-pass centroid copy and table, the bounds with the refine counter right
-// behind them (cleared together), and the list of rows for the float64 pass.
+// per-pass centroid copies and table, the bounds with the list counters right
+// behind them (cleared together), and the lists of rows for the float64
+// passes: two-candidate rows {h, row, c1, c2}, full-scan rows per head.
 struct TcWs {
   float* xn;
   bf16* cb;
   int2* table;
+  float* centT;
   Bounds* bd;
-  int* refine_count;
-  int* refine;
+  int* counts;  // [0] two-candidate rows, [1 + h] full-scan rows of head h
+  int4* list2;
+  int* list_full;  // [H][N]
 };
+
+static size_t zeroed_bytes(int H) { return sizeof(Bounds) * H + sizeof(int) * ((size_t)H + 1); }
 
 static size_t tc_layout(int H, int N, int d, int C, TcWs* out, void* ws) {
   Carve cv(ws);
@@ -510,9 +671,12 @@ static size_t tc_layout(int H, int N, int d, int C, TcWs* out, void* ws) {
   w.xn = cv.take<float>((size_t)H * N);
   w.cb = cv.take<bf16>((size_t)H * Cr * d);
   w.table = cv.take<int2>((size_t)H * Cpad);
-  w.bd = cv.take<Bounds>((size_t)H + 1);
-  w.refine_count = reinterpret_cast<int*>(w.bd ? w.bd + H : nullptr);
-  w.refine = cv.take<int>((size_t)H * N * kRefineInts);
+  w.centT = cv.take<float>((size_t)H * d * C);
+  char* z = cv.take<char>(zeroed_bytes(H));
+  w.bd = reinterpret_cast<Bounds*>(z);
+  w.counts = z ? reinterpret_cast<int*>(z + sizeof(Bounds) * H) : nullptr;
+  w.list2 = cv.take<int4>((size_t)H * N);
+  w.list_full = cv.take<int>((size_t)H * N);
   if (out) *out = w;
   return cv.used();
 }
@@ -553,7 +717,7 @@ static cudaError_t assign_launch(const bf16* X, int H, int N, int C, const float
   const int stages = pick_stages(D, C);
   int nbits = 1;
   while ((1 << nbits) < Cpad) ++nbits;
-  k_prep_centroids<D><<<dim3(Cr / 8, H), 256, 0, st>>>(cent, C, Cpad, Cr, w.cb, w.table, w.bd);
+  k_prep_centroids<D><<<dim3(Cr / 32, H), 256, 0, st>>>(cent, C, Cpad, Cr, w.cb, w.table, w.centT, w.bd);
   note_launch();
   CUtensorMap tmx, tmc;
   if (!tma_map_bf16_3d(&tmx, X, D, N, H, BM) || !tma_map_bf16_3d(&tmc, w.cb, D, Cr, H, 128))
@@ -564,10 +728,15 @@ static cudaError_t assign_launch(const bf16* X, int H, int N, int C, const float
   const int T = (N + BM - 1) / BM;
   const int tpc = pick_tiles_per_cta(H, T);
   k_assign_tc<D><<<dim3((T + tpc - 1) / tpc, H), kThreads, smem, st>>>(
-      tmx, tmc, w.table, w.bd, w.xn, N, Cpad, Cr, stages, tpc, nbits, labels, w.refine, w.refine_count,
-      status_word());
+      tmx, tmc, w.table, w.bd, w.xn, N, Cpad, Cr, stages, tpc, nbits, labels, w.list2, w.list_full,
+      w.counts, status_word());
   note_launch();
-  k_refine<D><<<148 * 4, 256, 0, st>>>(X, cent, N, C, w.refine, w.refine_count, labels);
+  k_refine2<D><<<148 * 4, 256, 0, st>>>(X, cent, N, C, w.list2, w.counts, labels);
+  note_launch();
+  const int fthreads = C > kFullThreads ? kFullThreads : (C + 31) / 32 * 32;
+  const int fgx = std::max(1, (148 * 8 + H - 1) / H);
+  k_refine_full<D><<<dim3(fgx, H), fthreads, 0, st>>>(X, cent, w.centT, N, C, w.list_full, w.counts + 1,
+                                                       labels);
   note_launch();
   return cudaGetLastError();
 }
@@ -576,7 +745,7 @@ cudaError_t kmeans_assign_tc(const void* Xv, int H, int N, int d, int C, const f
                              int32_t* labels, void* ws, cudaStream_t st) {
   TcWs w;
   tc_layout(H, N, d, C, &w, ws);
-  cudaError_t e = cudaMemsetAsync(w.bd, 0, sizeof(Bounds) * ((size_t)H + 1), st);
+  cudaError_t e = cudaMemsetAsync(w.bd, 0, zeroed_bytes(H), st);
   if (e != cudaSuccess) return e;
   const bf16* X = static_cast<const bf16*>(Xv);
   if (d == 128) return assign_launch<128>(X, H, N, C, cent, labels, w, st);

@@ -27,43 +27,50 @@ __global__ void k_chunk_hist(const int32_t* __restrict__ labels, int N, int C, i
   for (int c = threadIdx.x; c < C; c += blockDim.x) out[(size_t)c * nchunk] = hist[c];
 }
 
-// One block per head: exclusive scan over the head's C*nchunk entries.
-__global__ void k_scan(int32_t* __restrict__ bh, int C, int nchunk, int N,
-                       int32_t* __restrict__ counts, int32_t* __restrict__ offsets) {
+// One block per head: exclusive scan over the head's C*nchunk entries, in
+// tiles of 4 consecutive entries per thread (coalesced) with a running carry.
+__global__ void __launch_bounds__(1024) k_scan(int32_t* __restrict__ bh, int C, int nchunk, int N,
+                                               int32_t* __restrict__ counts, int32_t* __restrict__ offsets) {
   __shared__ int32_t warp_tot[32];
   const int h = blockIdx.x;
   const long long M = (long long)C * nchunk;
   int32_t* a = bh + (size_t)h * M;
-  const int T = blockDim.x;
-  const long long per = (M + T - 1) / T;
-  const long long beg = per * threadIdx.x, end = min(M, beg + per);
-  int32_t s = 0;
-  for (long long i = beg; i < end; ++i) s += a[i];
-  // block exclusive scan of s
+  const int T = blockDim.x, nw = T >> 5;
   const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
-  int32_t v = s;
-  for (int o = 1; o < 32; o <<= 1) {
-    int32_t u = __shfl_up_sync(0xffffffffu, v, o);
-    if (lane >= o) v += u;
-  }
-  if (lane == 31) warp_tot[w] = v;
-  __syncthreads();
-  if (w == 0) {
-    int32_t t = (lane < (T >> 5)) ? warp_tot[lane] : 0;
+  int32_t carry = 0;
+  for (long long t0 = 0; t0 < M; t0 += 4LL * T) {
+    const long long i0 = t0 + 4LL * threadIdx.x;
+    int32_t x[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) x[k] = (i0 + k < M) ? a[i0 + k] : 0;
+    const int32_t s = x[0] + x[1] + x[2] + x[3];
+    int32_t v = s;  // inclusive warp scan
+#pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
-      int32_t u = __shfl_up_sync(0xffffffffu, t, o);
-      if (lane >= o) t += u;
+      const int32_t u = __shfl_up_sync(0xffffffffu, v, o);
+      if (lane >= o) v += u;
     }
-    warp_tot[lane] = t;  // inclusive
+    if (lane == 31) warp_tot[w] = v;
+    __syncthreads();
+    if (w == 0) {
+      int32_t t = lane < nw ? warp_tot[lane] : 0;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int32_t u = __shfl_up_sync(0xffffffffu, t, o);
+        if (lane >= o) t += u;
+      }
+      warp_tot[lane] = t;  // inclusive over warps
+    }
+    __syncthreads();
+    int32_t run = carry + v - s + (w > 0 ? warp_tot[w - 1] : 0);
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      if (i0 + k < M) a[i0 + k] = run;
+      run += x[k];
+    }
+    carry += warp_tot[nw - 1];
+    __syncthreads();
   }
-  __syncthreads();
-  int32_t run = v - s + (w > 0 ? warp_tot[w - 1] : 0);
-  for (long long i = beg; i < end; ++i) {
-    int32_t x = a[i];
-    a[i] = run;
-    run += x;
-  }
-  __syncthreads();
   int32_t* off = offsets + (size_t)h * (C + 1);
   for (int c = threadIdx.x; c < C; c += T) off[c] = a[(size_t)c * nchunk];
   if (threadIdx.x == 0) off[C] = N;
