@@ -105,7 +105,7 @@ FwdLayout layout(const svgear_params* p, void* ws) {
   L.exec_pairs = cv.take<int64_t>(H);
   size_t sb = kmeans_ws_bytes(H, Nq, d, Cq);
   sb = std::max(sb, kmeans_ws_bytes(H, Nk, d, Ck));
-  sb = std::max(sb, block_error_ws_bytes(H, Cq, Ck));
+  sb = std::max(sb, block_error_ws_bytes(H, Cq, Ck, d, p->dtype));
   sb = std::max(sb, attn_ws_bytes(H, Nq, Nk, d, Cq, Ck));
   L.scratch = cv.take<char>(sb);
   L.scratch_bytes = sb;
@@ -191,7 +191,7 @@ int svgear_permute(const void* X, int dtype, const int32_t* labels, int H, int N
 
 size_t svgear_block_error_workspace_size(const svgear_params* p) {
   if (check_params(p)) return 0;
-  return block_error_ws_bytes(p->H, p->Cq, p->Ck);
+  return block_error_ws_bytes(p->H, p->Cq, p->Ck, p->d, p->dtype);
 }
 
 int svgear_block_error(const float* Qbar, const float* Kbar, const float* Vbar, const void* Kp,
@@ -202,7 +202,7 @@ int svgear_block_error(const float* Qbar, const float* Kbar, const float* Vbar, 
   if (r) return r;
   if (!Qbar || !Kbar || !Kp || !k_off || !key_scalars || !E || !M) return SVGEAR_ERR_INVALID;
   if (!aligned16(Qbar) || !aligned16(Kbar) || !aligned16(Kp)) return SVGEAR_ERR_INVALID;
-  if (!ws || ws_bytes < block_error_ws_bytes(p->H, p->Cq, p->Ck)) return SVGEAR_ERR_WORKSPACE;
+  if (!ws || ws_bytes < block_error_ws_bytes(p->H, p->Cq, p->Ck, p->d, p->dtype)) return SVGEAR_ERR_WORKSPACE;
   return cuda_status(block_error_run(Qbar, Kbar, Vbar, Kp, Vp, k_off, key_scalars, p->dtype, p->H,
                                      p->Nk, p->d, p->Cq, p->Ck, eff_scale(p), E, M, ws, S(stream)));
 }

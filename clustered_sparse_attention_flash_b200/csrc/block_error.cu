@@ -23,38 +23,52 @@ namespace svg {
 
 namespace {
 
-// L[a][c] = s qbar_a.kbar_c (float64 dot, stored float32) and
-// M[a] = max over non-empty c of L[a][c].  One block per (a, head).
+// L[a][c] = s qbar_a.kbar_c (float64 dot, stored float32) for a tile of
+// 32 query centroids x 32 key centroids per block (both staged in shared
+// memory); each thread owns one query centroid and four key centroids.
 template <int D>
 __global__ void __launch_bounds__(256) k_centroid_logits(const float* __restrict__ Qbar,
-                                                         const float* __restrict__ Kbar,
-                                                         const int32_t* __restrict__ k_off, int Cq,
-                                                         int Ck, float scale, float* __restrict__ L,
-                                                         float* __restrict__ M) {
-  __shared__ float q[D];
-  __shared__ float red[32];
-  const int h = blockIdx.y, a = blockIdx.x;
-  for (int t = threadIdx.x; t < D; t += blockDim.x) q[t] = Qbar[((size_t)h * Cq + a) * D + t];
+                                                         const float* __restrict__ Kbar, int Cq, int Ck,
+                                                         float scale, float* __restrict__ L) {
+  __shared__ float qs[32][D + 1];
+  __shared__ float ks[32][D + 1];
+  const int h = blockIdx.z, a0 = blockIdx.y * 32, c0 = blockIdx.x * 32;
+  for (int e = threadIdx.x; e < 32 * D; e += blockDim.x) {
+    const int r = e / D, t = e % D;
+    qs[r][t] = a0 + r < Cq ? Qbar[((size_t)h * Cq + a0 + r) * D + t] : 0.f;
+    ks[r][t] = c0 + r < Ck ? Kbar[((size_t)h * Ck + c0 + r) * D + t] : 0.f;
+  }
   __syncthreads();
+  const int ar = threadIdx.x & 31, cg = threadIdx.x >> 5;  // query row, group of 4 key rows
+  double acc[4] = {0.0, 0.0, 0.0, 0.0};
+#pragma unroll 4
+  for (int t = 0; t < D; ++t) {
+    const double q = qs[ar][t];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) acc[i] = fma(q, (double)ks[cg * 4 + i][t], acc[i]);
+  }
+  const int a = a0 + ar;
+  if (a < Cq)
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int c = c0 + cg * 4 + i;
+      if (c < Ck) L[((size_t)h * Cq + a) * Ck + c] = (float)(acc[i] * (double)scale);
+    }
+}
+
+// M[a] = max over non-empty c of L[a][c]: one warp per (a, head).
+__global__ void __launch_bounds__(256) k_logit_max(const float* __restrict__ L, const int32_t* __restrict__ k_off,
+                                                   int H, int Cq, int Ck, float* __restrict__ M) {
+  const int row = blockIdx.x * 8 + (threadIdx.x >> 5), lane = threadIdx.x & 31;
+  if (row >= H * Cq) return;
+  const int h = row / Cq;
   const int32_t* off = k_off + (size_t)h * (Ck + 1);
+  const float* Lr = L + (size_t)row * Ck;
   float mx = -INFINITY;
-  for (int c = threadIdx.x; c < Ck; c += blockDim.x) {
-    const float* kb = Kbar + ((size_t)h * Ck + c) * D;
-    double acc = 0.0;
-#pragma unroll 8
-    for (int t = 0; t < D; ++t) acc = fma((double)q[t], (double)kb[t], acc);
-    const float l = (float)(acc * (double)scale);
-    L[((size_t)h * Cq + a) * Ck + c] = l;
-    if (off[c + 1] > off[c]) mx = fmaxf(mx, l);
-  }
+  for (int c = lane; c < Ck; c += 32)
+    if (off[c + 1] > off[c]) mx = fmaxf(mx, Lr[c]);
   for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = mx;
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    float m = -INFINITY;
-    for (int w = 0; w < (int)(blockDim.x >> 5); ++w) m = fmaxf(m, red[w]);
-    M[(size_t)h * Cq + a] = m;
-  }
+  if (lane == 0) M[row] = mx;
 }
 
 // One block per (key cluster c, head); thread t owns query cluster a = t (+128k).
@@ -131,18 +145,28 @@ __global__ void __launch_bounds__(128) k_block_error(const float* __restrict__ Q
 
 }  // namespace
 
-size_t block_error_ws_bytes(int H, int Cq, int Ck) {
-  return align_up((size_t)H * Cq * Ck * sizeof(float), 256);
+size_t block_error_ws_bytes(int H, int Cq, int Ck, int d, int dtype) {
+  size_t n = align_up((size_t)H * Cq * Ck * sizeof(float), 256);
+  // reserved whenever the shape allows the tensor-core kernel (no device query here)
+  if (block_error_tc_shape_ok(dtype, d, Cq)) n += align_up(block_error_tc_ws_bytes(H, d), 256);
+  return n;
 }
 
 cudaError_t block_error_run(const float* Qbar, const float* Kbar, const float* Vbar,
                             const void* Kp, const void* Vp, const int32_t* k_off,
                             const float* key_scalars, int dtype, int H, int Nk, int d, int Cq,
-                            int Ck, float scale, float* E, float* M, void* ws, cudaStream_t st) {
+                            int Ck, float scale, float* E, float* M, void* ws, cudaStream_t st,
+                            bool allow_tc) {
   (void)Vbar; (void)Vp;  // their contribution enters through key_scalars
   float* L = static_cast<float*>(ws);
-  if (d == 128) { k_centroid_logits<128><<<dim3(Cq, H), 256, 0, st>>>(Qbar, Kbar, k_off, Cq, Ck, scale, L, M); note_launch(); }
-  else { k_centroid_logits<64><<<dim3(Cq, H), 256, 0, st>>>(Qbar, Kbar, k_off, Cq, Ck, scale, L, M); note_launch(); }
+  const dim3 lg((Ck + 31) / 32, (Cq + 31) / 32, H);
+  if (d == 128) { k_centroid_logits<128><<<lg, 256, 0, st>>>(Qbar, Kbar, Cq, Ck, scale, L); note_launch(); }
+  else { k_centroid_logits<64><<<lg, 256, 0, st>>>(Qbar, Kbar, Cq, Ck, scale, L); note_launch(); }
+  k_logit_max<<<(H * Cq + 7) / 8, 256, 0, st>>>(L, k_off, H, Cq, Ck, M); note_launch();
+  if (allow_tc && block_error_tc_supported(dtype, d, Cq, Nk)) {
+    char* qhl = static_cast<char*>(ws) + align_up((size_t)H * Cq * Ck * sizeof(float), 256);
+    return block_error_tc_run(Qbar, Kp, k_off, key_scalars, L, M, H, Nk, d, Cq, Ck, scale, E, qhl, st);
+  }
   dim3 g(Ck, H);
   if (dtype == DT_BF16) {
     if (d == 128) { k_block_error<bf16, 128><<<g, 128, 0, st>>>(Qbar, Kbar, static_cast<const bf16*>(Kp), k_off, key_scalars, L, M, H, Nk, Cq, Ck, scale, E); note_launch(); }
@@ -198,7 +222,8 @@ extern "C" int svgear_block_error_noalloc(const float* Qbar, const float* Kbar, 
   float* L = noalloc_scratch(&e);
   if (!L) return SVGEAR_ERR_CUDA;
   const float scale = p->scale > 0.f ? p->scale : 1.0f / sqrtf((float)p->d);
+  // the static scratch holds the centroid logits only: CUDA-core block error
   e = block_error_run(Qbar, Kbar, Vbar, Kp, Vp, k_off, key_scalars, p->dtype, p->H, p->Nk, p->d, p->Cq,
-                      p->Ck, scale, E, M, L, static_cast<cudaStream_t>(stream));
+                      p->Ck, scale, E, M, L, static_cast<cudaStream_t>(stream), false);
   return e == cudaSuccess ? SVGEAR_OK : SVGEAR_ERR_CUDA;
 }

@@ -39,11 +39,21 @@ cudaError_t value_stats(const void* Vp, int dtype, const int32_t* off, int H, in
                         int C, float* Vbar, float* key_scalars, cudaStream_t st);
 
 // ---- block error
-size_t block_error_ws_bytes(int H, int Cq, int Ck);
+// Workspace: centroid logits [H,Cq,Ck] float, then (tensor-core path) the
+// hi/lo query-centroid operand.
+size_t block_error_ws_bytes(int H, int Cq, int Ck, int d, int dtype);
 cudaError_t block_error_run(const float* Qbar, const float* Kbar, const float* Vbar,
                             const void* Kp, const void* Vp, const int32_t* k_off,
                             const float* key_scalars, int dtype, int H, int Nk, int d, int Cq,
-                            int Ck, float scale, float* E, float* M, void* ws, cudaStream_t st);
+                            int Ck, float scale, float* E, float* M, void* ws, cudaStream_t st,
+                            bool allow_tc = true);
+// tensor-core kernel (block_error_tc.cu); L and M already computed
+bool block_error_tc_shape_ok(int dtype, int d, int Cq);
+bool block_error_tc_supported(int dtype, int d, int Cq, int Nk);
+size_t block_error_tc_ws_bytes(int H, int d);
+cudaError_t block_error_tc_run(const float* Qbar, const void* Kp, const int32_t* k_off, const float* ks,
+                               const float* L, const float* M, int H, int Nk, int d, int Cq, int Ck,
+                               float scale, float* E, void* ws, cudaStream_t st);
 
 // ---- routing
 cudaError_t route_run(const float* E, const int32_t* k_counts, const int32_t* q_counts,
