@@ -6,39 +6,39 @@
 //       / [ the same without v ],
 // written to row perm_q[i] of the output.
 //
-// One block per unit of two 128-row query tiles (A, B) of one query cluster;
-// units never straddle clusters, so both tiles share one key stream, read
-// once per block:
+// One block per 128-row query tile of one query cluster (tiles never straddle
+// clusters, so a tile has one key stream):
 //   * exact part: the rows of the routed clusters (routing order),
-//     concatenated and cut into 64-key tiles (the last one masked),
-//   * compensation part: all key centroids in 64-row tiles, logit bias
+//     concatenated and cut into 128-key tiles (the last one masked),
+//   * compensation part: all key centroids in 128-row tiles, logit bias
 //     log2|k_c| (in base-2 units) or -inf when c is routed or empty.  The
 //     float32 centroids enter as bf16 hi + lo pairs (two MMAs each for S and
 //     for P.V), so their rounding stays near 2^-17 instead of 2^-9; such a
 //     tile occupies two ring stages (hi, then lo).
-// Key tiles flow through a four-stage ring of 64-row K and V tiles.  Keys and
-// values are staged in an "8-row group" layout (each key cluster padded to a
-// multiple of 8 rows, each group of 8 rows stored as [16-byte chunk][row]),
-// which is directly a no-swizzle UMMA operand (K-major for K, MN-major for
-// V); a stage is therefore one or a few contiguous runs, each moved by a
-// single cp.async.bulk completing on the stage's mbarrier.  Padding rows are
-// masked through the stage's bias vector.
+// Keys and values are staged in an "8-row group" layout (each key cluster
+// padded to a multiple of 8 rows, each group of 8 rows stored as
+// [16-byte chunk][row]), which is directly a no-swizzle UMMA operand (K-major
+// for K, MN-major for V); a stage is one or a few contiguous runs, each moved
+// by a single cp.async.bulk.  K and V have separate two-slot rings: a K slot is
+// free once S of its tile is computed, a V slot (and the stage's bias vector)
+// once P.V is; padding rows are masked through the bias vector.
 // Warp roles (12 warps):
-//   warp 0      tensor-memory allocation, MMA issue (one thread): per key
-//               tile S_A, S_B = Q_{A,B} K^T into double-buffered S, then
-//               O_{A,B} += P V of the previous tile with P read from tensor
-//               memory;
-//   warps 1-3   load the two query tiles (cp.async into the 128-byte-swizzled
-//               layout), then produce every third key stage each (bulk copies
-//               issued by one lane, bias vectors by the whole warp);
-//   warps 4-7   softmax of tile A, warps 8-11 softmax of tile B (thread =
-//               query row): row max, lazy rescale of O when the max grows by
-//               more than 2^8, P = 2^(x - m) in bf16 written over the S
-//               columns it came from, final O / l and the permuted store.
-// Tensor memory (512 columns): S_A[0..1] [0,128), S_B[0..1] [128,256),
-// O_A [256,384), O_B [384,512); P_X[b] lives in the first 32 columns of S_X[b].
-// Every decision that guards a warp-collective tensor-memory access is made
-// warp-uniform, and every wait is time-bounded (device status word on expiry).
+//   warp 0      tensor-memory allocation, MMA issue (one thread): S = Q K^T
+//               into double-buffered S (N = 128 keys), then O += P V of the
+//               previous tile with P read from tensor memory;
+//   warps 1-3   load the query tile; warps 1 and 2 then produce the even
+//               and the odd stages (bulk copies issued by one lane, bias
+//               vectors by the warp);
+//   warps 4-7   softmax of keys 0..63 of every stage, warps 8-11 of keys
+//               64..127 (thread = query row): the two halves exchange their
+//               row maxima through shared memory, rescale O lazily (each its
+//               half of the d columns) when the maximum grows by more than 2^8,
+//               write P = 2^(x - m) in bf16 over the S columns of the stage
+//               and finally store O / l through perm_q.
+// Tensor memory (512 columns): S[0..1] [0,256), O [256,256+d); P[b] lives in
+// the first 64 columns of S[b].  Every decision that guards a warp-collective
+// tensor-memory access is made warp-uniform, and every wait is time-bounded
+// (device status word on expiry).
 #include <algorithm>
 #include <cmath>
 
@@ -50,15 +50,15 @@ namespace svg {
 
 namespace {
 
-constexpr int BQ = 128;        // rows per query tile (two tiles per block)
-constexpr int BN = 64;         // keys per ring stage
+constexpr int BQ = 128;        // rows per query tile (one tile per block)
+constexpr int BN = 128;        // keys per ring stage
 constexpr int kThreads = 384;
 constexpr int kProducers = 96;
-constexpr int kStages = 4;
-constexpr int kUnitRows = 2 * BQ;
+constexpr int kSlots = 2;      // K ring and V ring
+constexpr int kUnitRows = BQ;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr uint32_t kColS = 0, kColO = 256;
-constexpr int kMaxRanges = 1024;  // routed clusters staged in shared memory
+constexpr int kMaxRanges = 512;  // routed clusters staged in shared memory
 
 __device__ __forceinline__ float ex2(float x) {
   float y;
@@ -79,8 +79,8 @@ __host__ __device__ __forceinline__ size_t g8_offset(size_t row, int chunk) {
 }
 
 // bf16 hi/lo copies of the key / value centroids (x = hi + lo + O(2^-17 x)),
-// in the 8-row group layout with rows padded to a multiple of 64 (zeros),
-// and log2 of the cluster sizes (-inf for empty or padding).
+// in the 8-row group layout with rows padded to a multiple of the stage size
+// (zeros), and log2 of the cluster sizes (-inf for empty or padding).
 template <int D>
 __global__ void k_prep_comp(const float* __restrict__ Kbar, const float* __restrict__ Vbar,
                             const int32_t* __restrict__ k_off, int Ck, int Ckpad, uint8_t* __restrict__ kh,
@@ -166,7 +166,7 @@ __global__ void k_pack(const bf16* __restrict__ Kp, const bf16* __restrict__ Vp,
   }
 }
 
-// Per head: (query cluster, first row) of every 256-row unit.
+// Per head: (query cluster, first row) of every 128-row query tile.
 __global__ void k_tile_table_tc(const int32_t* __restrict__ q_off, int Cq, int tmax,
                                 int2* __restrict__ tiles, int32_t* __restrict__ ntiles) {
   __shared__ int32_t wtot[32];
@@ -211,18 +211,22 @@ __global__ void k_tile_table_tc(const int32_t* __restrict__ q_off, int Cq, int t
 
 template <int D>
 struct AttnSmem {
-  static constexpr int kQTile = BQ * D * 2;   // one 128-row bf16 query tile
-  static constexpr int kKTile = BN * D * 2;   // one 64-row bf16 key (or value) tile
-  static constexpr int q_off = 0;             // [2] query tiles
-  static constexpr int k_off = q_off + 2 * kQTile;
-  static constexpr int v_off = k_off + kStages * kKTile;
-  static constexpr int bias_off = v_off + kStages * kKTile;
-  static constexpr int flag_off = bias_off + kStages * BN * 4;
+  static constexpr int kQTile = BQ * D * 2;   // the 128-row bf16 query tile
+  static constexpr int kKTile = BN * D * 2;   // one 128-row bf16 key (or value) tile
+  static constexpr int q_off = 0;
+  static constexpr int k_off = q_off + kQTile;                       // [kSlots] key tiles
+  static constexpr int v_off = k_off + kSlots * kKTile;              // [kSlots] value tiles
+  static constexpr int bias_off = v_off + kSlots * kKTile;           // [kSlots][BN] log2 biases
+  static constexpr int mx_off = bias_off + kSlots * BN * 4;          // [2 stages][2 halves][BQ] row maxima
+  static constexpr int ls_off = mx_off + 2 * 2 * BQ * 4;             // [2 halves][BQ] row sums
+  static constexpr int flag_off = ls_off + 2 * BQ * 4;               // [kSlots]: 1 = apply bias
   static constexpr int bits_off = flag_off + 64;
-  static constexpr int rng_off = bits_off + kMaxCkBits / 8;   // [3][kMaxRanges] start, prefix, len
-  static constexpr int pc_off = rng_off + 3 * kMaxRanges * 4 + 16;  // [producer warp][8] piece lists
-  static constexpr int bar_off = pc_off + 3 * 8 * 4 * 4;
-  static constexpr int total = bar_off + 40 * 8 + 1024;
+  static constexpr int rng_off = bits_off + kMaxCkBits / 8;          // [3][kMaxRanges] start, prefix, len
+  static constexpr int pc_off = rng_off + 3 * kMaxRanges * 4 + 16;   // [producer warp][16] piece lists
+  static constexpr int bar_off = pc_off + 3 * 16 * 16;
+  // at least 120 KB, so that one block (and one 512-column tensor-memory
+  // allocation) lives on an SM
+  static constexpr int total = bar_off + 32 * 8 + 1024 > 120 * 1024 ? bar_off + 32 * 8 + 1024 : 120 * 1024;
 };
 
 template <int D>
@@ -237,14 +241,17 @@ __global__ void __launch_bounds__(kThreads, 1)
               const int32_t* __restrict__ ntiles, int tmax, int Nq, int Nk, int Cq, int Ck, int Ckpad,
               float scale2, bf16* __restrict__ O, int* status) {
   using S = AttnSmem<D>;
-  constexpr int CPR = D / 8;  // 16-byte chunks per row
+  constexpr int CPR = D / 8;              // 16-byte chunks per row
   constexpr uint32_t kGroup = 8 * D * 2;  // bytes of one 8-row group
+  constexpr int kMaxPieces = 16;          // runs per stage (each at least 8 padded rows)
   const int h = blockIdx.y;
   if ((int)blockIdx.x >= ntiles[h]) return;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  float* bias_s = reinterpret_cast<float*>(smem + S::bias_off);   // [stage][BN] log2 biases
-  int* flag_s = reinterpret_cast<int*>(smem + S::flag_off);       // [stage]: 1 = apply bias
+  float* bias_s = reinterpret_cast<float*>(smem + S::bias_off);
+  float* mx_s = reinterpret_cast<float*>(smem + S::mx_off);
+  float* ls_s = reinterpret_cast<float*>(smem + S::ls_off);
+  int* flag_s = reinterpret_cast<int*>(smem + S::flag_off);
   uint32_t* bits = reinterpret_cast<uint32_t*>(smem + S::bits_off);
   int* rng_start = reinterpret_cast<int*>(smem + S::rng_off);  // first padded row of routed range i
   int* rng_cum = rng_start + kMaxRanges;                        // padded rows in ranges [0, i)
@@ -252,20 +259,22 @@ __global__ void __launch_bounds__(kThreads, 1)
   int4* pieces = reinterpret_cast<int4*>(smem + S::pc_off);     // stage row group, global row, groups, valid
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + S::bar_off);
   uint64_t* q_full = bars + 0;
-  uint64_t* kv_full = bars + 1;    // [kStages]
-  uint64_t* kv_empty = bars + 5;   // [kStages]
-  uint64_t* s_full = bars + 9;     // [tile X][2]
-  uint64_t* p_full = bars + 13;    // [tile X][2]
-  uint64_t* o_done = bars + 17;    // [tile X][2]
-  uint64_t* done = bars + 21;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 22);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 23);
+  uint64_t* k_full = bars + 1;     // [kSlots]
+  uint64_t* k_empty = bars + 3;    // [kSlots]
+  uint64_t* v_full = bars + 5;     // [kSlots]
+  uint64_t* v_empty = bars + 7;    // [kSlots]
+  uint64_t* s_full = bars + 9;     // [2]
+  uint64_t* p_full = bars + 11;    // [2]
+  uint64_t* o_done = bars + 13;    // [2]
+  uint64_t* mx_bar = bars + 15;    // [2]: both halves posted their row maxima
+  uint64_t* l_bar = bars + 17;     // both halves posted their row sums
+  uint64_t* done = bars + 18;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 19);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 20);
 
   const int2 unit = tiles[(size_t)h * tmax + blockIdx.x];
   const int a = unit.x, r0 = unit.y;
   const int qend = q_off[(size_t)h * (Cq + 1) + a + 1];
-  const bool has_b = r0 + BQ < qend;   // tile B holds at least one row of the cluster
-  const int ntq = has_b ? 2 : 1;
   const int ns = n_sel[(size_t)h * Cq + a];
   const int32_t* sl = sel + ((size_t)h * Cq + a) * Ck;
   const int32_t* koff = k_off + (size_t)h * (Ck + 1);
@@ -275,15 +284,19 @@ __global__ void __launch_bounds__(kThreads, 1)
   for (int i = threadIdx.x; i < (Ck + 31) / 32; i += blockDim.x) bits[i] = 0;
   if (threadIdx.x == 0) {
     tc::mbar_init(q_full, kProducers);
-    for (int i = 0; i < kStages; ++i) {
-      tc::mbar_init(kv_full + i, 1);  // one arrival carrying the stage's byte count
-      tc::mbar_init(kv_empty + i, 1);
+    for (int i = 0; i < kSlots; ++i) {
+      tc::mbar_init(k_full + i, 1);   // one arrival carrying the stage's byte count
+      tc::mbar_init(k_empty + i, 1);
+      tc::mbar_init(v_full + i, 1);
+      tc::mbar_init(v_empty + i, 1);
     }
-    for (int i = 0; i < 4; ++i) {
+    for (int i = 0; i < 2; ++i) {
       tc::mbar_init(s_full + i, 1);
-      tc::mbar_init(p_full + i, 128);
+      tc::mbar_init(p_full + i, 256);
       tc::mbar_init(o_done + i, 1);
+      tc::mbar_init(mx_bar + i, 256);
     }
+    tc::mbar_init(l_bar, 256);
     tc::mbar_init(done, 1);
     *abort_flag = 0;
     tc::mbar_fence_init();
@@ -343,49 +356,47 @@ __global__ void __launch_bounds__(kThreads, 1)
       // descriptors are built once; a K step only moves the start-address
       // field (address >> 4): +2 per 32 B inside a swizzled row, +1024 per
       // 16 KB region of Q, +16 per 256 B of a K tile, +2*kGroup/16 for V
-      uint64_t qd[2];
-      for (int x = 0; x < 2; ++x) qd[x] = tc::desc_kmajor(tc::smem_u32(smem + S::q_off + x * S::kQTile), BQ * 128u, 0);
+      const uint64_t qd = tc::desc_kmajor(tc::smem_u32(smem + S::q_off), BQ * 128u, 0);
       const uint64_t kd0 = tc::desc_kmajor_g8(tc::smem_u32(smem + S::k_off), kGroup, 0);
       const uint64_t vd0 = tc::desc_mnmajor_g8(tc::smem_u32(smem + S::v_off), kGroup, 0);
       constexpr uint64_t kStageStep = (uint64_t)(S::kKTile >> 4);
       bool ok = tc::mbar_wait(q_full, 0, abort_flag, status);
       auto issue_pv = [&](int j) -> bool {
         const int b = j & 1, u0 = ustart(j), np = nparts(j);
-        for (int x = 0; x < ntq; ++x) {
-          if (!tc::mbar_wait(p_full + x * 2 + b, (j >> 1) & 1, abort_flag, status)) return false;
-          tc::tc_fence_after();
-          const uint32_t pcol = tmem + kColS + (uint32_t)(x * 128 + b * 64);
-          const uint32_t ocol = tmem + kColO + (uint32_t)x * 128u;
-          for (int p = 0; p < np; ++p) {
-            const uint64_t vd = vd0 + (uint64_t)((u0 + p) % kStages) * kStageStep;
+        for (int p = 0; p < np; ++p)
+          if (!tc::mbar_wait(v_full + (u0 + p) % kSlots, ((u0 + p) / kSlots) & 1, abort_flag, status)) return false;
+        if (!tc::mbar_wait(p_full + b, (j >> 1) & 1, abort_flag, status)) return false;
+        tc::tc_fence_after();
+        const uint32_t pcol = tmem + kColS + (uint32_t)(b * 128);
+        const uint32_t ocol = tmem + kColO;
+        for (int p = 0; p < np; ++p) {
+          const uint64_t vd = vd0 + (uint64_t)((u0 + p) % kSlots) * kStageStep;
 #pragma unroll
-            for (int k = 0; k < BN / 16; ++k)
-              tc::mma_ts(ocol, pcol + (uint32_t)k * 8u, vd + (uint64_t)k * (2u * kGroup >> 4), id_o,
-                         (j > 0 || p > 0 || k > 0) ? 1u : 0u);
-          }
-          tc::mma_commit(o_done + x * 2 + b);
+          for (int k = 0; k < BN / 16; ++k)
+            tc::mma_ts(ocol, pcol + (uint32_t)k * 8u, vd + (uint64_t)k * (2u * kGroup >> 4), id_o,
+                       (j > 0 || p > 0 || k > 0) ? 1u : 0u);
         }
-        for (int p = 0; p < np; ++p) tc::mma_commit(kv_empty + (u0 + p) % kStages);
+        tc::mma_commit(o_done + b);
+        for (int p = 0; p < np; ++p) tc::mma_commit(v_empty + (u0 + p) % kSlots);
         return true;
       };
       for (int j = 0; ok && j < ntile; ++j) {
         const int b = j & 1, u0 = ustart(j), np = nparts(j);
         for (int p = 0; ok && p < np; ++p)
-          ok = tc::mbar_wait(kv_full + (u0 + p) % kStages, ((u0 + p) / kStages) & 1, abort_flag, status);
+          ok = tc::mbar_wait(k_full + (u0 + p) % kSlots, ((u0 + p) / kSlots) & 1, abort_flag, status);
         if (!ok) break;
         tc::tc_fence_after();
-        // S_X[b] was last read as P_X[b] by P.V of tile j-2, issued before
-        for (int x = 0; x < ntq; ++x) {
-          const uint32_t scol = tmem + kColS + (uint32_t)(x * 128 + b * 64);
-          for (int p = 0; p < np; ++p) {
-            const uint64_t kd = kd0 + (uint64_t)((u0 + p) % kStages) * kStageStep;
+        // S[b] was last read as P[b] by P.V of tile j-2, issued before
+        const uint32_t scol = tmem + kColS + (uint32_t)(b * 128);
+        for (int p = 0; p < np; ++p) {
+          const uint64_t kd = kd0 + (uint64_t)((u0 + p) % kSlots) * kStageStep;
 #pragma unroll
-            for (int k = 0; k < D / 16; ++k)
-              tc::mma_ss(scol, qd[x] + (uint64_t)((k >> 2) * 1024 + (k & 3) * 2), kd + (uint64_t)k * 16u, id_s,
-                         (p > 0 || k > 0) ? 1u : 0u);
-          }
-          tc::mma_commit(s_full + x * 2 + b);
+          for (int k = 0; k < D / 16; ++k)
+            tc::mma_ss(scol, qd + (uint64_t)((k >> 2) * 1024 + (k & 3) * 2), kd + (uint64_t)k * 16u, id_s,
+                       (p > 0 || k > 0) ? 1u : 0u);
         }
+        tc::mma_commit(s_full + b);
+        for (int p = 0; p < np; ++p) tc::mma_commit(k_empty + (u0 + p) % kSlots);
         if (j > 0 && !issue_pv(j - 1)) { ok = false; break; }
       }
       if (ok && ntile > 0) issue_pv(ntile - 1);
@@ -397,14 +408,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int pt = threadIdx.x - 32;
     {
       const bf16* Qh = Qp + (size_t)h * Nq * D;
-      for (int x = 0; x < 2; ++x) {
-        const uint32_t qa = tc::smem_u32(smem + S::q_off + x * S::kQTile);
-        for (int e = pt; e < BQ * CPR; e += kProducers) {
-          const int r = e / CPR, c = e % CPR, row = r0 + x * BQ + r;
-          const bool valid = row < qend;
-          tc::cp_async16(qa + tc::sw128_offset(r, c, BQ), Qh + (size_t)(valid ? row : 0) * D + c * 8,
-                         valid ? 16u : 0u);
-        }
+      const uint32_t qa = tc::smem_u32(smem + S::q_off);
+      for (int e = pt; e < BQ * CPR; e += kProducers) {
+        const int r = e / CPR, c = e % CPR, row = r0 + r;
+        const bool valid = row < qend;
+        tc::cp_async16(qa + tc::sw128_offset(r, c, BQ), Qh + (size_t)(valid ? row : 0) * D + c * 8,
+                       valid ? 16u : 0u);
       }
       tc::cp_async_wait_all();
       tc::fence_proxy_async();
@@ -412,19 +421,20 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     asm volatile("bar.sync 2, 96;" ::: "memory");  // range prefix ready
     {
-      // the three producer warps (one per scheduler they share with softmax
-      // warps) build and issue every third stage
+      // one producer warp per ring slot (warp 1: even stages, warp 2: odd
+      // stages; warp 3 only helps with the query tile), so that the waits on a
+      // slot's barriers come in order and never run a phase ahead: keys once
+      // the K slot is free, values, bias and mask once the V slot is
       const int pw = warp - 1;
-      int4* pcs = pieces + pw * 8;  // this warp's piece list
+      int4* pcs = pieces + pw * kMaxPieces;  // this warp's piece list
       const uint8_t* Kh = kpk + (size_t)h * npad * D * 2;
       const uint8_t* Vh = vpk + (size_t)h * npad * D * 2;
       const float* LC = lc2 + (size_t)h * Ckpad;
       const size_t cbase = (size_t)h * Ckpad * D * 2;
       const int nstage = ustart(ntile);  // total ring stages of the stream
       const unsigned rot = n_ex > 0 ? (blockIdx.x * 2654435761u + h * 40503u) % (unsigned)n_ex : 0u;
-      for (int u = pw; u < nstage; u += 3) {
-        const int st = u % kStages;
-        if (!tc::mbar_wait_warp(kv_empty + st, ((u / kStages) & 1) ^ 1, abort_flag, status)) break;
+      for (int u = pw; pw < kSlots && u < nstage; u += kSlots) {
+        const int st = u % kSlots;
         const bool exact = u < n_ex;
         int j = exact ? u : n_ex + (u - n_ex) / 2;
         const int p = exact ? 0 : (u - n_ex) & 1;
@@ -432,12 +442,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         // softmax does not depend on the order), so that the blocks of a head
         // do not all read the same popular clusters at the same time
         if (exact) j = (int)(((unsigned)j + rot) % (unsigned)n_ex);
-        float* bias = bias_s + st * BN;
         const uint32_t ka = tc::smem_u32(smem + S::k_off + st * S::kKTile);
         const uint32_t va = tc::smem_u32(smem + S::v_off + st * S::kKTile);
+        int npc = 0, tail = BN;
+        uint32_t okm = 0, bytes = 0;
+        // ---- keys
+        if (!tc::mbar_wait_warp(k_empty + st, ((u / kSlots) & 1) ^ 1, abort_flag, status)) break;
         if (exact) {
           // pieces of the padded routed stream in [j*BN, j*BN + BN)
-          int npc = 0, tail = BN;
           if (lane == 0) {
             const int pos0 = j * BN, end = pos0 + BN;
             int ri;
@@ -453,7 +465,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             int cum = ns <= kMaxRanges ? rng_cum[ri] : 0;
             int pos = pos0;
-            while (pos < end && ri < ns && npc < 8) {
+            while (pos < end && ri < ns && npc < kMaxPieces) {
               int pst, len;
               if (ri < kMaxRanges) {
                 pst = rng_start[ri]; len = rng_len[ri];
@@ -470,10 +482,47 @@ __global__ void __launch_bounds__(kThreads, 1)
               ++ri;
             }
             tail = pos - pos0;
+            // a piece must stay inside the stage tile and the packed rows;
+            // one that does not is dropped (status word) instead of copied
+            for (int q = 0; q < npc; ++q) {
+              const int4 pc = pcs[q];
+              const bool good = pc.x >= 0 && pc.z > 0 && pc.x + pc.z <= BN / 8 && pc.y >= 0 &&
+                                (size_t)pc.y + (size_t)pc.z * 8 <= npad;
+              if (good) { okm |= 1u << q; bytes += (uint32_t)pc.z * kGroup; }
+              else set_status(status, ST_BOUNDS);
+            }
           }
           npc = __shfl_sync(0xffffffffu, npc, 0);
           tail = __shfl_sync(0xffffffffu, tail, 0);
           __syncwarp();
+          // zero the key rows past the stream end so the MMAs see finite values
+          if (tail < BN) {
+            uint4* kz = reinterpret_cast<uint4*>(smem + S::k_off + st * S::kKTile) + (tail >> 3) * (kGroup / 16);
+            const int nz = ((BN - tail) >> 3) * (int)(kGroup / 16);
+            for (int i = lane; i < nz; i += 32) kz[i] = make_uint4(0, 0, 0, 0);
+            tc::fence_proxy_async();
+          }
+          __syncwarp();
+          if (lane == 0) {
+            tc::mbar_arrive_expect_tx(k_full + st, bytes);
+            for (int q = 0; q < npc; ++q) {
+              if (!((okm >> q) & 1u)) continue;
+              const int4 pc = pcs[q];
+              tc::bulk_g2s(ka + (uint32_t)pc.x * kGroup, Kh + (size_t)(pc.y >> 3) * kGroup,
+                           (uint32_t)pc.z * kGroup, k_full + st);
+            }
+          }
+        } else if (lane == 0) {
+          const uint32_t n = (uint32_t)(BN / 8) * kGroup;
+          const size_t go = cbase + (size_t)(((j - n_ex) * BN) >> 3) * kGroup;
+          tc::mbar_arrive_expect_tx(k_full + st, n);
+          tc::bulk_g2s(ka, (p == 0 ? kb_hi : kb_lo) + go, n, k_full + st);
+        }
+        __syncwarp();
+        // ---- values, bias and mask
+        if (!tc::mbar_wait_warp(v_empty + st, ((u / kSlots) & 1) ^ 1, abort_flag, status)) break;
+        float* bias = bias_s + st * BN;
+        if (exact) {
           // bias: valid keys 0, padding and the stream tail -inf
           for (int i = lane; i < BN; i += 32) bias[i] = -INFINITY;
           __syncwarp();
@@ -481,52 +530,39 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int4 pc = pcs[q];
             for (int i = lane; i < pc.w; i += 32) bias[pc.x * 8 + i] = 0.f;
           }
-          // zero the rows past the stream end so the MMAs see finite values
           if (tail < BN) {
-            uint4* kz = reinterpret_cast<uint4*>(smem + S::k_off + st * S::kKTile) + (tail >> 3) * (kGroup / 16);
             uint4* vz = reinterpret_cast<uint4*>(smem + S::v_off + st * S::kKTile) + (tail >> 3) * (kGroup / 16);
             const int nz = ((BN - tail) >> 3) * (int)(kGroup / 16);
-            for (int i = lane; i < nz; i += 32) { kz[i] = make_uint4(0, 0, 0, 0); vz[i] = make_uint4(0, 0, 0, 0); }
+            for (int i = lane; i < nz; i += 32) vz[i] = make_uint4(0, 0, 0, 0);
             tc::fence_proxy_async();
           }
           if (lane == 0) flag_s[st] = 1;
           __syncwarp();
           if (lane == 0) {
-            // a piece must stay inside the stage tile and the packed rows;
-            // one that does not is dropped (status word) instead of copied
-            uint32_t okm = 0, bytes = 0;
-            for (int q = 0; q < npc; ++q) {
-              const int4 pc = pcs[q];
-              const bool good = pc.x >= 0 && pc.z > 0 && pc.x + pc.z <= BN / 8 && pc.y >= 0 &&
-                                (size_t)pc.y + (size_t)pc.z * 8 <= npad;
-              if (good) { okm |= 1u << q; bytes += 2u * (uint32_t)pc.z * kGroup; }
-              else set_status(status, ST_BOUNDS);
-            }
-            tc::mbar_arrive_expect_tx(kv_full + st, bytes);
+            tc::mbar_arrive_expect_tx(v_full + st, bytes);
             for (int q = 0; q < npc; ++q) {
               if (!((okm >> q) & 1u)) continue;
               const int4 pc = pcs[q];
-              const uint32_t n = (uint32_t)pc.z * kGroup;
-              const size_t go = (size_t)(pc.y >> 3) * kGroup;
-              tc::bulk_g2s(ka + (uint32_t)pc.x * kGroup, Kh + go, n, kv_full + st);
-              tc::bulk_g2s(va + (uint32_t)pc.x * kGroup, Vh + go, n, kv_full + st);
+              tc::bulk_g2s(va + (uint32_t)pc.x * kGroup, Vh + (size_t)(pc.y >> 3) * kGroup,
+                           (uint32_t)pc.z * kGroup, v_full + st);
             }
           }
         } else {
           const int c0 = (j - n_ex) * BN;
-          for (int i = lane; i < BN; i += 32) {
-            const int c = c0 + i;
-            const bool routed = c < Ck && ((bits[c >> 5] >> (c & 31)) & 1u);
-            bias[i] = routed ? -INFINITY : LC[c];
+          if (p == 0) {
+            for (int i = lane; i < BN; i += 32) {
+              const int c = c0 + i;
+              const bool routed = c < Ck && ((bits[c >> 5] >> (c & 31)) & 1u);
+              bias[i] = routed ? -INFINITY : LC[c];
+            }
+            if (lane == 0) flag_s[st] = 1;
           }
-          if (lane == 0) flag_s[st] = 1;
           __syncwarp();
           if (lane == 0) {
             const uint32_t n = (uint32_t)(BN / 8) * kGroup;
             const size_t go = cbase + (size_t)(c0 >> 3) * kGroup;
-            tc::mbar_arrive_expect_tx(kv_full + st, 2u * n);
-            tc::bulk_g2s(ka, (p == 0 ? kb_hi : kb_lo) + go, n, kv_full + st);
-            tc::bulk_g2s(va, (p == 0 ? vb_hi : vb_lo) + go, n, kv_full + st);
+            tc::mbar_arrive_expect_tx(v_full + st, n);
+            tc::bulk_g2s(va, (p == 0 ? vb_hi : vb_lo) + go, n, v_full + st);
           }
         }
         __syncwarp();
@@ -534,21 +570,23 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else {
     // -------------------------------------------------------------- softmax
-    const int x = (warp - 4) >> 2;            // query tile A (0) or B (1)
+    const int half = (warp - 4) >> 2;         // keys [64 half, 64 half + 64) of every stage
     const int r = ((warp & 3) << 5) + lane;   // tile row == TMEM lane
     const uint32_t lane_base = (uint32_t)((warp & 3) << 5) << 16;
-    const uint32_t scol = kColS + (uint32_t)x * 128u, ocol = kColO + (uint32_t)x * 128u;
+    constexpr int OH = D / 2;                 // columns of O per half
+    const uint32_t ocol = kColO + (uint32_t)(half * OH);
     float m_used = -INFINITY, l = 0.f;
-    bool ok = x < ntq;
+    bool ok = true;
     for (int j = 0; ok && j < ntile; ++j) {
-      const int u0 = ustart(j), st = u0 % kStages, b = j & 1;
-      if (!tc::mbar_wait_warp(s_full + x * 2 + b, (j >> 1) & 1, abort_flag, status)) { ok = false; break; }
+      const int u0 = ustart(j), st = u0 % kSlots, b = j & 1;
+      const uint32_t scol = kColS + (uint32_t)(b * 128);
+      if (!tc::mbar_wait_warp(s_full + b, (j >> 1) & 1, abort_flag, status)) { ok = false; break; }
       tc::tc_fence_after();
-      float xs[BN];
+      float xs[64];
       {
         uint32_t v0[32], v1[32];
-        tc::tmem_ld32(tmem + lane_base + scol + (uint32_t)(b * 64), v0);
-        tc::tmem_ld32(tmem + lane_base + scol + (uint32_t)(b * 64 + 32), v1);
+        tc::tmem_ld32(tmem + lane_base + scol + (uint32_t)(half * 64), v0);
+        tc::tmem_ld32(tmem + lane_base + scol + (uint32_t)(half * 64 + 32), v1);
         tc::tmem_ld_wait();
 #pragma unroll
         for (int i = 0; i < 32; ++i) {
@@ -557,37 +595,49 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
       // bias / mask of this stage: acquire the producers' writes through the
-      // stage's full barrier (its next phase needs this tile's P first)
-      if (!tc::mbar_wait_warp(kv_full + st, (u0 / kStages) & 1, abort_flag, status)) { ok = false; break; }
+      // stage's V barrier (its next phase needs this tile's P.V first)
+      if (!tc::mbar_wait_warp(v_full + st, (u0 / kSlots) & 1, abort_flag, status)) { ok = false; break; }
       if (flag_s[st]) {
-        const float* bias = bias_s + st * BN;
+        const float* bias = bias_s + st * BN + half * 64;
 #pragma unroll
-        for (int i = 0; i < BN; i += 4) {
+        for (int i = 0; i < 64; i += 4) {
           const float4 b4 = *reinterpret_cast<const float4*>(bias + i);
           xs[i] += b4.x; xs[i + 1] += b4.y; xs[i + 2] += b4.z; xs[i + 3] += b4.w;
         }
       }
       float mx;
-      {  // 8 independent chains instead of one 64-long chain
+      {  // eight independent chains of three-input maxima
         float m8[8];
 #pragma unroll
-        for (int k = 0; k < 8; ++k) m8[k] = xs[k];
+        for (int k = 0; k < 8; ++k) m8[k] = fmaxf(xs[k], xs[8 + k]);
 #pragma unroll
-        for (int i = 8; i < BN; ++i) m8[i & 7] = fmaxf(m8[i & 7], xs[i]);
-        mx = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])), fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
+        for (int i = 16; i < 64; i += 16)
+#pragma unroll
+          for (int k = 0; k < 8; ++k) m8[k] = tc::fmax3(m8[k], xs[i + k], xs[i + 8 + k]);
+        mx = fmaxf(tc::fmax3(m8[0], m8[1], m8[2]), tc::fmax3(tc::fmax3(m8[3], m8[4], m8[5]), m8[6], m8[7]));
       }
+      // the row maximum over both halves (this also orders both halves' reads
+      // of S before either writes P over it)
+      float* mxp = mx_s + (j & 1) * 2 * BQ;
+      mxp[half * BQ + r] = mx;
+      tc::tc_fence_before();
+      tc::mbar_arrive(mx_bar + (j & 1));
+      if (!tc::mbar_wait_warp(mx_bar + (j & 1), (j >> 1) & 1, abort_flag, status)) { ok = false; break; }
+      tc::tc_fence_after();
+      mx = fmaxf(mx, mxp[(1 - half) * BQ + r]);
       // lazy rescale: a row whose maximum grew by more than 2^8 rescales O and
-      // l.  The tensor-memory accesses are warp-collective, so the warp
-      // rescales together (factor 1 for rows that do not need it).
+      // l (each half its d/2 columns of O).  The tensor-memory accesses are
+      // warp-collective, so the warp rescales together (factor 1 for rows that
+      // do not need it).
       const bool grow = mx > m_used + 8.f;
       const bool has_o = j > 0 && m_used > -INFINITY;
       if (__any_sync(0xffffffffu, grow && has_o)) {
         const int pb = (j - 1) & 1;
-        if (!tc::mbar_wait_warp(o_done + x * 2 + pb, ((j - 1) >> 1) & 1, abort_flag, status)) { ok = false; break; }
+        if (!tc::mbar_wait_warp(o_done + pb, ((j - 1) >> 1) & 1, abort_flag, status)) { ok = false; break; }
         tc::tc_fence_after();
         const float f = (grow && has_o) ? ex2(m_used - mx) : 1.f;
 #pragma unroll
-        for (int q = 0; q < D / 16; ++q) {
+        for (int q = 0; q < OH / 16; ++q) {
           uint32_t ov[16];
           tc::tmem_ld16(tmem + lane_base + ocol + (uint32_t)q * 16u, ov);
           tc::tmem_ld_wait();
@@ -602,7 +652,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const float mref = m_used == -INFINITY ? 0.f : m_used;
       float r8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-      for (int q = 0; q < BN / 32; ++q) {
+      for (int q = 0; q < 2; ++q) {
         uint32_t pk[16];
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
@@ -610,27 +660,33 @@ __global__ void __launch_bounds__(kThreads, 1)
           r8[i & 7] += p0 + p1;
           pk[i] = pack_bf16(p0, p1);
         }
-        // P over the first 32 columns of this S buffer (already read above)
-        tc::tmem_st16(tmem + lane_base + scol + (uint32_t)(b * 64 + q * 16), pk);
+        // P (bf16 pairs) over the first 64 columns of this S buffer: keys
+        // 64 half + 32 q + [0, 32) in columns 32 half + 16 q + [0, 16)
+        tc::tmem_st16(tmem + lane_base + scol + (uint32_t)(half * 32 + q * 16), pk);
       }
       tc::tmem_st_wait();
       l += ((r8[0] + r8[1]) + (r8[2] + r8[3])) + ((r8[4] + r8[5]) + (r8[6] + r8[7]));
       tc::tc_fence_before();
-      tc::mbar_arrive(p_full + x * 2 + b);
+      tc::mbar_arrive(p_full + b);
     }
-    // epilogue: wait for the last P.V of this tile, normalise, store via perm_q
+    // epilogue: both halves' row sums, the last P.V, normalise, store via perm_q
+    if (ok) {
+      ls_s[half * BQ + r] = l;
+      tc::mbar_arrive(l_bar);
+      ok = tc::mbar_wait_warp(l_bar, 0, abort_flag, status);
+    }
     if (ok && ntile > 0) {
       const int jl = ntile - 1;
-      ok = tc::mbar_wait_warp(o_done + x * 2 + (jl & 1), (jl >> 1) & 1, abort_flag, status);
+      ok = tc::mbar_wait_warp(o_done + (jl & 1), (jl >> 1) & 1, abort_flag, status);
     }
     if (ok && ntile > 0) {
       tc::tc_fence_after();
-      const int row = r0 + x * BQ + r;
+      const int row = r0 + r;
       const bool valid = row < qend;
-      const float inv = 1.f / l;
-      bf16* orow = O + ((size_t)h * Nq + (valid ? perm_q[(size_t)h * Nq + row] : 0)) * D;
+      const float inv = 1.f / (ls_s[r] + ls_s[BQ + r]);
+      bf16* orow = O + ((size_t)h * Nq + (valid ? perm_q[(size_t)h * Nq + row] : 0)) * D + half * OH;
 #pragma unroll
-      for (int q = 0; q < D / 16; ++q) {
+      for (int q = 0; q < OH / 16; ++q) {
         uint32_t ov[16];
         tc::tmem_ld16(tmem + lane_base + ocol + (uint32_t)q * 16u, ov);
         tc::tmem_ld_wait();
@@ -661,7 +717,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
-int round64(int x) { return (x + 63) / 64 * 64; }
+int round_stage(int x) { return (x + BN - 1) / BN * BN; }
 
 struct AttnWs {
   uint8_t *kh, *kl, *vh, *vl, *kpk, *vpk;
@@ -674,7 +730,7 @@ struct AttnWs {
 
 size_t attn_layout(int H, int Nq, int Nk, int d, int Cq, int Ck, AttnWs* out, void* ws) {
   Carve cv(ws);
-  const int Ckpad = round64(Ck);
+  const int Ckpad = round_stage(Ck);
   const int tmax = (Nq + kUnitRows - 1) / kUnitRows + Cq;
   AttnWs w;
   w.npad = (size_t)Nk + 8 * (size_t)Ck;  // rows after padding every cluster to 8
@@ -699,7 +755,7 @@ cudaError_t launch(const void* Qp, const void* Kp, const void* Vp, const int32_t
                    void* ws, cudaStream_t st) {
   AttnWs w;
   attn_layout(H, Nq, Nk, D, Cq, Ck, &w, ws);
-  const int Ckpad = round64(Ck);
+  const int Ckpad = round_stage(Ck);
   const int tmax = (Nq + kUnitRows - 1) / kUnitRows + Cq;
   k_prep_comp<D><<<dim3(Ckpad, H), 64, 0, st>>>(Kbar, Vbar, k_off, Ck, Ckpad, w.kh, w.kl, w.vh, w.vl, w.lc2);
   note_launch();
