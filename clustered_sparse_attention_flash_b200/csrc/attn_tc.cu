@@ -217,8 +217,8 @@ struct AttnSmem {
   static constexpr int k_off = q_off + kQTile;                       // [kSlots] key tiles
   static constexpr int v_off = k_off + kSlots * kKTile;              // [kSlots] value tiles
   static constexpr int bias_off = v_off + kSlots * kKTile;           // [kSlots][BN] log2 biases
-  static constexpr int mx_off = bias_off + kSlots * BN * 4;          // [2 stages][2 halves][BQ] row maxima
-  static constexpr int ls_off = mx_off + 2 * 2 * BQ * 4;             // [2 halves][BQ] row sums
+  static constexpr int mx_off = bias_off + kSlots * BN * 4;          // [2 groups][BQ] row maxima
+  static constexpr int ls_off = mx_off + 2 * 2 * BQ * 4;             // [2 groups][BQ] row sums
   static constexpr int flag_off = ls_off + 2 * BQ * 4;               // [kSlots]: 1 = apply bias
   static constexpr int bits_off = flag_off + 64;
   static constexpr int rng_off = bits_off + kMaxCkBits / 8;          // [3][kMaxRanges] start, prefix, len
@@ -266,8 +266,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* s_full = bars + 9;     // [2]
   uint64_t* p_full = bars + 11;    // [2]
   uint64_t* o_done = bars + 13;    // [2]
-  uint64_t* mx_bar = bars + 15;    // [2]: both halves posted their row maxima
-  uint64_t* l_bar = bars + 17;     // both halves posted their row sums
+  uint64_t* l_bar = bars + 17;     // both softmax groups posted their row maxima and sums
   uint64_t* done = bars + 18;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 19);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 20);
@@ -292,9 +291,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int i = 0; i < 2; ++i) {
       tc::mbar_init(s_full + i, 1);
-      tc::mbar_init(p_full + i, 256);
+      tc::mbar_init(p_full + i, 128);
       tc::mbar_init(o_done + i, 1);
-      tc::mbar_init(mx_bar + i, 256);
     }
     tc::mbar_init(l_bar, 256);
     tc::mbar_init(done, 1);
@@ -368,13 +366,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!tc::mbar_wait(p_full + b, (j >> 1) & 1, abort_flag, status)) return false;
         tc::tc_fence_after();
         const uint32_t pcol = tmem + kColS + (uint32_t)(b * 128);
-        const uint32_t ocol = tmem + kColO;
+        const uint32_t ocol = tmem + kColO + (uint32_t)(b * D);  // O[b]: the stages of softmax group b
         for (int p = 0; p < np; ++p) {
           const uint64_t vd = vd0 + (uint64_t)((u0 + p) % kSlots) * kStageStep;
 #pragma unroll
           for (int k = 0; k < BN / 16; ++k)
             tc::mma_ts(ocol, pcol + (uint32_t)k * 8u, vd + (uint64_t)k * (2u * kGroup >> 4), id_o,
-                       (j > 0 || p > 0 || k > 0) ? 1u : 0u);
+                       (j > 1 || p > 0 || k > 0) ? 1u : 0u);
         }
         tc::mma_commit(o_done + b);
         for (int p = 0; p < np; ++p) tc::mma_commit(v_empty + (u0 + p) % kSlots);
@@ -570,74 +568,61 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else {
     // -------------------------------------------------------------- softmax
-    const int half = (warp - 4) >> 2;         // keys [64 half, 64 half + 64) of every stage
+    // group w (warps 4-7: w = 0, warps 8-11: w = 1) takes the stages j with
+    // j % 2 == w: S[w], its own running maximum m_w, row sum l_w and
+    // accumulator O[w]; the two partial results are merged at the end.
+    const int w = (warp - 4) >> 2;
     const int r = ((warp & 3) << 5) + lane;   // tile row == TMEM lane
     const uint32_t lane_base = (uint32_t)((warp & 3) << 5) << 16;
-    constexpr int OH = D / 2;                 // columns of O per half
-    const uint32_t ocol = kColO + (uint32_t)(half * OH);
+    const uint32_t scol = kColS + (uint32_t)(w * 128);
+    const uint32_t ocol = kColO + (uint32_t)(w * D);
     float m_used = -INFINITY, l = 0.f;
     bool ok = true;
-    for (int j = 0; ok && j < ntile; ++j) {
-      const int u0 = ustart(j), st = u0 % kSlots, b = j & 1;
-      const uint32_t scol = kColS + (uint32_t)(b * 128);
-      if (!tc::mbar_wait_warp(s_full + b, (j >> 1) & 1, abort_flag, status)) { ok = false; break; }
-      tc::tc_fence_after();
-      float xs[64];
-      {
-        uint32_t v0[32], v1[32];
-        tc::tmem_ld32(tmem + lane_base + scol + (uint32_t)(half * 64), v0);
-        tc::tmem_ld32(tmem + lane_base + scol + (uint32_t)(half * 64 + 32), v1);
-        tc::tmem_ld_wait();
-#pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          xs[i] = __uint_as_float(v0[i]) * scale2;
-          xs[32 + i] = __uint_as_float(v1[i]) * scale2;
-        }
-      }
+    for (int j = w; ok && j < ntile; j += 2) {
+      const int u0 = ustart(j), st = u0 % kSlots;
+      if (!tc::mbar_wait_warp(s_full + w, (j >> 1) & 1, abort_flag, status)) { ok = false; break; }
       // bias / mask of this stage: acquire the producers' writes through the
-      // stage's V barrier (its next phase needs this tile's P.V first)
+      // stage's V barrier (its next phase needs this stage's P.V first)
       if (!tc::mbar_wait_warp(v_full + st, (u0 / kSlots) & 1, abort_flag, status)) { ok = false; break; }
-      if (flag_s[st]) {
-        const float* bias = bias_s + st * BN + half * 64;
-#pragma unroll
-        for (int i = 0; i < 64; i += 4) {
-          const float4 b4 = *reinterpret_cast<const float4*>(bias + i);
-          xs[i] += b4.x; xs[i + 1] += b4.y; xs[i + 2] += b4.z; xs[i + 3] += b4.w;
-        }
-      }
-      float mx;
-      {  // eight independent chains of three-input maxima
+      tc::tc_fence_after();
+      const float* bias = bias_s + st * BN;
+      // pass 1: the row maximum over the stage's 128 keys, 64 at a time
+      float mx = -INFINITY;
+#pragma unroll 1
+      for (int h2 = 0; h2 < 2; ++h2) {
+        uint32_t v[64];
+        tc::tmem_ld32(tmem + lane_base + scol + (uint32_t)(h2 * 64), *reinterpret_cast<uint32_t(*)[32]>(v));
+        tc::tmem_ld32(tmem + lane_base + scol + (uint32_t)(h2 * 64 + 32), *reinterpret_cast<uint32_t(*)[32]>(v + 32));
+        tc::tmem_ld_wait();
         float m8[8];
 #pragma unroll
-        for (int k = 0; k < 8; ++k) m8[k] = fmaxf(xs[k], xs[8 + k]);
+        for (int k = 0; k < 8; ++k) m8[k] = -INFINITY;
 #pragma unroll
-        for (int i = 16; i < 64; i += 16)
+        for (int i = 0; i < 64; i += 16) {
+          const float4 b0 = *reinterpret_cast<const float4*>(bias + h2 * 64 + i);
+          const float4 b1 = *reinterpret_cast<const float4*>(bias + h2 * 64 + i + 4);
+          const float4 b2 = *reinterpret_cast<const float4*>(bias + h2 * 64 + i + 8);
+          const float4 b3 = *reinterpret_cast<const float4*>(bias + h2 * 64 + i + 12);
+          const float bb[16] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w,
+                                b2.x, b2.y, b2.z, b2.w, b3.x, b3.y, b3.z, b3.w};
 #pragma unroll
-          for (int k = 0; k < 8; ++k) m8[k] = tc::fmax3(m8[k], xs[i + k], xs[i + 8 + k]);
-        mx = fmaxf(tc::fmax3(m8[0], m8[1], m8[2]), tc::fmax3(tc::fmax3(m8[3], m8[4], m8[5]), m8[6], m8[7]));
+          for (int k = 0; k < 8; ++k)
+            m8[k] = tc::fmax3(m8[k], fmaf(__uint_as_float(v[i + k]), scale2, bb[k]),
+                              fmaf(__uint_as_float(v[i + 8 + k]), scale2, bb[8 + k]));
+        }
+        mx = fmaxf(mx, fmaxf(tc::fmax3(m8[0], m8[1], m8[2]), tc::fmax3(tc::fmax3(m8[3], m8[4], m8[5]), m8[6], m8[7])));
       }
-      // the row maximum over both halves (this also orders both halves' reads
-      // of S before either writes P over it)
-      float* mxp = mx_s + (j & 1) * 2 * BQ;
-      mxp[half * BQ + r] = mx;
-      tc::tc_fence_before();
-      tc::mbar_arrive(mx_bar + (j & 1));
-      if (!tc::mbar_wait_warp(mx_bar + (j & 1), (j >> 1) & 1, abort_flag, status)) { ok = false; break; }
-      tc::tc_fence_after();
-      mx = fmaxf(mx, mxp[(1 - half) * BQ + r]);
-      // lazy rescale: a row whose maximum grew by more than 2^8 rescales O and
-      // l (each half its d/2 columns of O).  The tensor-memory accesses are
-      // warp-collective, so the warp rescales together (factor 1 for rows that
-      // do not need it).
+      // lazy rescale: a row whose maximum grew by more than 2^8 rescales O[w]
+      // and l_w.  The tensor-memory accesses are warp-collective, so the warp
+      // rescales together (factor 1 for rows that do not need it).
       const bool grow = mx > m_used + 8.f;
-      const bool has_o = j > 0 && m_used > -INFINITY;
+      const bool has_o = j >= 2 && m_used > -INFINITY;
       if (__any_sync(0xffffffffu, grow && has_o)) {
-        const int pb = (j - 1) & 1;
-        if (!tc::mbar_wait_warp(o_done + pb, ((j - 1) >> 1) & 1, abort_flag, status)) { ok = false; break; }
+        if (!tc::mbar_wait_warp(o_done + w, ((j >> 1) - 1) & 1, abort_flag, status)) { ok = false; break; }
         tc::tc_fence_after();
         const float f = (grow && has_o) ? ex2(m_used - mx) : 1.f;
 #pragma unroll
-        for (int q = 0; q < OH / 16; ++q) {
+        for (int q = 0; q < D / 16; ++q) {
           uint32_t ov[16];
           tc::tmem_ld16(tmem + lane_base + ocol + (uint32_t)q * 16u, ov);
           tc::tmem_ld_wait();
@@ -650,55 +635,82 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       if (grow) m_used = mx;
       const float mref = m_used == -INFINITY ? 0.f : m_used;
+      // pass 2: P = 2^(x - m) in bf16 over the first 64 columns of S[w]
+      // (keys 64 h2 + [0, 64) in columns 32 h2 + [0, 32), after they are read)
       float r8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+#pragma unroll 1
+      for (int h2 = 0; h2 < 2; ++h2) {
+        uint32_t v[64];
+        tc::tmem_ld32(tmem + lane_base + scol + (uint32_t)(h2 * 64), *reinterpret_cast<uint32_t(*)[32]>(v));
+        tc::tmem_ld32(tmem + lane_base + scol + (uint32_t)(h2 * 64 + 32), *reinterpret_cast<uint32_t(*)[32]>(v + 32));
+        tc::tmem_ld_wait();
 #pragma unroll
-      for (int q = 0; q < 2; ++q) {
-        uint32_t pk[16];
+        for (int q = 0; q < 2; ++q) {
+          uint32_t pk[16];
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          const float p0 = ex2(xs[q * 32 + 2 * i] - mref), p1 = ex2(xs[q * 32 + 2 * i + 1] - mref);
-          r8[i & 7] += p0 + p1;
-          pk[i] = pack_bf16(p0, p1);
+          for (int i = 0; i < 16; i += 2) {
+            const float4 b4 = *reinterpret_cast<const float4*>(bias + h2 * 64 + q * 32 + 2 * i);
+            const int c = q * 32 + 2 * i;
+            const float p0 = ex2(fmaf(__uint_as_float(v[c]), scale2, b4.x) - mref);
+            const float p1 = ex2(fmaf(__uint_as_float(v[c + 1]), scale2, b4.y) - mref);
+            const float p2 = ex2(fmaf(__uint_as_float(v[c + 2]), scale2, b4.z) - mref);
+            const float p3 = ex2(fmaf(__uint_as_float(v[c + 3]), scale2, b4.w) - mref);
+            r8[i & 7] += p0 + p1;
+            r8[(i + 1) & 7] += p2 + p3;
+            pk[i] = pack_bf16(p0, p1);
+            pk[i + 1] = pack_bf16(p2, p3);
+          }
+          tc::tmem_st16(tmem + lane_base + scol + (uint32_t)(h2 * 32 + q * 16), pk);
         }
-        // P (bf16 pairs) over the first 64 columns of this S buffer: keys
-        // 64 half + 32 q + [0, 32) in columns 32 half + 16 q + [0, 16)
-        tc::tmem_st16(tmem + lane_base + scol + (uint32_t)(half * 32 + q * 16), pk);
       }
       tc::tmem_st_wait();
       l += ((r8[0] + r8[1]) + (r8[2] + r8[3])) + ((r8[4] + r8[5]) + (r8[6] + r8[7]));
       tc::tc_fence_before();
-      tc::mbar_arrive(p_full + b);
+      tc::mbar_arrive(p_full + w);
     }
-    // epilogue: both halves' row sums, the last P.V, normalise, store via perm_q
+    // epilogue: merge the two groups' (m, l, O), normalise, store via perm_q.
+    // Group w writes the columns [w d/2, w d/2 + d/2) of the output rows.
     if (ok) {
-      ls_s[half * BQ + r] = l;
+      mx_s[w * BQ + r] = m_used;
+      ls_s[w * BQ + r] = l;
       tc::mbar_arrive(l_bar);
       ok = tc::mbar_wait_warp(l_bar, 0, abort_flag, status);
     }
-    if (ok && ntile > 0) {
-      const int jl = ntile - 1;
-      ok = tc::mbar_wait_warp(o_done + (jl & 1), (jl >> 1) & 1, abort_flag, status);
+    // the last P.V into each accumulator
+    for (int x = 0; ok && x < 2; ++x) {
+      const int jl = ntile - 1 - ((ntile - 1 - x) & 1);  // last stage with j % 2 == x
+      if (jl >= 0) ok = tc::mbar_wait_warp(o_done + x, (jl >> 1) & 1, abort_flag, status);
     }
-    if (ok && ntile > 0) {
+    if (ok) {
       tc::tc_fence_after();
+      const float m0 = mx_s[r], m1 = mx_s[BQ + r];
+      const float mm = fmaxf(m0, m1);
+      // a group that saw no key (or no stage) contributes nothing; its
+      // accumulator is not read
+      const bool u0ok = m0 > -INFINITY, u1ok = m1 > -INFINITY;
+      const float a0 = u0ok ? ex2(m0 - mm) : 0.f, a1 = u1ok ? ex2(m1 - mm) : 0.f;
+      const float lt = ls_s[r] * a0 + ls_s[BQ + r] * a1;
+      const float inv = lt > 0.f ? 1.f / lt : 0.f;
+      const float f0 = a0 * inv, f1 = a1 * inv;
       const int row = r0 + r;
       const bool valid = row < qend;
-      const float inv = 1.f / (ls_s[r] + ls_s[BQ + r]);
-      bf16* orow = O + ((size_t)h * Nq + (valid ? perm_q[(size_t)h * Nq + row] : 0)) * D + half * OH;
+      constexpr int OH = D / 2;
+      bf16* orow = O + ((size_t)h * Nq + (valid ? perm_q[(size_t)h * Nq + row] : 0)) * D + w * OH;
 #pragma unroll
       for (int q = 0; q < OH / 16; ++q) {
-        uint32_t ov[16];
-        tc::tmem_ld16(tmem + lane_base + ocol + (uint32_t)q * 16u, ov);
+        uint32_t o0[16], o1[16];
+        tc::tmem_ld16(tmem + lane_base + kColO + (uint32_t)(w * OH + q * 16), o0);
+        tc::tmem_ld16(tmem + lane_base + kColO + (uint32_t)(D + w * OH + q * 16), o1);
         tc::tmem_ld_wait();
+        float o[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i)
+          o[i] = (u0ok ? __uint_as_float(o0[i]) * f0 : 0.f) + (u1ok ? __uint_as_float(o1[i]) * f1 : 0.f);
         uint4 w0, w1;
-        w0.x = pack_bf16(__uint_as_float(ov[0]) * inv, __uint_as_float(ov[1]) * inv);
-        w0.y = pack_bf16(__uint_as_float(ov[2]) * inv, __uint_as_float(ov[3]) * inv);
-        w0.z = pack_bf16(__uint_as_float(ov[4]) * inv, __uint_as_float(ov[5]) * inv);
-        w0.w = pack_bf16(__uint_as_float(ov[6]) * inv, __uint_as_float(ov[7]) * inv);
-        w1.x = pack_bf16(__uint_as_float(ov[8]) * inv, __uint_as_float(ov[9]) * inv);
-        w1.y = pack_bf16(__uint_as_float(ov[10]) * inv, __uint_as_float(ov[11]) * inv);
-        w1.z = pack_bf16(__uint_as_float(ov[12]) * inv, __uint_as_float(ov[13]) * inv);
-        w1.w = pack_bf16(__uint_as_float(ov[14]) * inv, __uint_as_float(ov[15]) * inv);
+        w0.x = pack_bf16(o[0], o[1]); w0.y = pack_bf16(o[2], o[3]);
+        w0.z = pack_bf16(o[4], o[5]); w0.w = pack_bf16(o[6], o[7]);
+        w1.x = pack_bf16(o[8], o[9]); w1.y = pack_bf16(o[10], o[11]);
+        w1.z = pack_bf16(o[12], o[13]); w1.w = pack_bf16(o[14], o[15]);
         if (valid) {
           reinterpret_cast<uint4*>(orow + q * 16)[0] = w0;
           reinterpret_cast<uint4*>(orow + q * 16)[1] = w1;
