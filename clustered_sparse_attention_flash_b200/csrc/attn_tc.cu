@@ -55,6 +55,8 @@ constexpr int BN = 128;        // keys per ring stage
 constexpr int kThreads = 384;
 constexpr int kProducers = 96;
 constexpr int kSlots = 2;      // K ring and V ring
+constexpr int kKSlots = kSlots;
+constexpr int kVSlots = kSlots;
 constexpr int kUnitRows = BQ;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr uint32_t kColS = 0, kColO = 256;
@@ -214,16 +216,16 @@ struct AttnSmem {
   static constexpr int kQTile = BQ * D * 2;   // the 128-row bf16 query tile
   static constexpr int kKTile = BN * D * 2;   // one 128-row bf16 key (or value) tile
   static constexpr int q_off = 0;
-  static constexpr int k_off = q_off + kQTile;                       // [kSlots] key tiles
-  static constexpr int v_off = k_off + kSlots * kKTile;              // [kSlots] value tiles
-  static constexpr int bias_off = v_off + kSlots * kKTile;           // [kSlots][BN] log2 biases
-  static constexpr int mx_off = bias_off + kSlots * BN * 4;          // [2 groups][BQ] row maxima
+  static constexpr int k_off = q_off + kQTile;                       // [kKSlots] key tiles
+  static constexpr int v_off = k_off + kKSlots * kKTile;             // [kVSlots] value tiles
+  static constexpr int bias_off = v_off + kVSlots * kKTile;          // [kVSlots][BN] log2 biases
+  static constexpr int mx_off = bias_off + kVSlots * BN * 4;         // [2 groups][BQ] row maxima
   static constexpr int ls_off = mx_off + 2 * 2 * BQ * 4;             // [2 groups][BQ] row sums
-  static constexpr int flag_off = ls_off + 2 * BQ * 4;               // [kSlots]: 1 = apply bias
+  static constexpr int flag_off = ls_off + 2 * BQ * 4;               // [kVSlots]: 1 = apply bias
   static constexpr int bits_off = flag_off + 64;
   static constexpr int rng_off = bits_off + kMaxCkBits / 8;          // [3][kMaxRanges] start, prefix, len
-  static constexpr int pc_off = rng_off + 3 * kMaxRanges * 4 + 16;   // [producer warp][16] piece lists
-  static constexpr int bar_off = pc_off + 3 * 16 * 16;
+  static constexpr int pc_off = rng_off + 3 * kMaxRanges * 4 + 16;   // [producer warp][32] piece lists
+  static constexpr int bar_off = pc_off + 2 * 32 * 16;
   // at least 120 KB, so that one block (and one 512-column tensor-memory
   // allocation) lives on an SM
   static constexpr int total = bar_off + 32 * 8 + 1024 > 120 * 1024 ? bar_off + 32 * 8 + 1024 : 120 * 1024;
@@ -243,7 +245,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   using S = AttnSmem<D>;
   constexpr int CPR = D / 8;              // 16-byte chunks per row
   constexpr uint32_t kGroup = 8 * D * 2;  // bytes of one 8-row group
-  constexpr int kMaxPieces = 16;          // runs per stage (each at least 8 padded rows)
+  constexpr int kMaxPieces = 32;          // runs per stage (one per lane)
   const int h = blockIdx.y;
   if ((int)blockIdx.x >= ntiles[h]) return;
   extern __shared__ uint8_t smem_raw[];
@@ -259,13 +261,13 @@ __global__ void __launch_bounds__(kThreads, 1)
   int4* pieces = reinterpret_cast<int4*>(smem + S::pc_off);     // stage row group, global row, groups, valid
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + S::bar_off);
   uint64_t* q_full = bars + 0;
-  uint64_t* k_full = bars + 1;     // [kSlots]
-  uint64_t* k_empty = bars + 3;    // [kSlots]
-  uint64_t* v_full = bars + 5;     // [kSlots]
-  uint64_t* v_empty = bars + 7;    // [kSlots]
-  uint64_t* s_full = bars + 9;     // [2]
-  uint64_t* p_full = bars + 11;    // [2]
-  uint64_t* o_done = bars + 13;    // [2]
+  uint64_t* k_full = bars + 1;     // [kKSlots]
+  uint64_t* k_empty = bars + 4;    // [kKSlots]
+  uint64_t* v_full = bars + 7;     // [kVSlots]
+  uint64_t* v_empty = bars + 9;    // [kVSlots]
+  uint64_t* s_full = bars + 11;    // [2]
+  uint64_t* p_full = bars + 13;    // [2]
+  uint64_t* o_done = bars + 15;    // [2]
   uint64_t* l_bar = bars + 17;     // both softmax groups posted their row maxima and sums
   uint64_t* done = bars + 18;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 19);
@@ -283,9 +285,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   for (int i = threadIdx.x; i < (Ck + 31) / 32; i += blockDim.x) bits[i] = 0;
   if (threadIdx.x == 0) {
     tc::mbar_init(q_full, kProducers);
-    for (int i = 0; i < kSlots; ++i) {
+    for (int i = 0; i < kKSlots; ++i) {
       tc::mbar_init(k_full + i, 1);   // one arrival carrying the stage's byte count
       tc::mbar_init(k_empty + i, 1);
+    }
+    for (int i = 0; i < kVSlots; ++i) {
       tc::mbar_init(v_full + i, 1);
       tc::mbar_init(v_empty + i, 1);
     }
@@ -362,39 +366,39 @@ __global__ void __launch_bounds__(kThreads, 1)
       auto issue_pv = [&](int j) -> bool {
         const int b = j & 1, u0 = ustart(j), np = nparts(j);
         for (int p = 0; p < np; ++p)
-          if (!tc::mbar_wait(v_full + (u0 + p) % kSlots, ((u0 + p) / kSlots) & 1, abort_flag, status)) return false;
+          if (!tc::mbar_wait(v_full + (u0 + p) % kVSlots, ((u0 + p) / kVSlots) & 1, abort_flag, status)) return false;
         if (!tc::mbar_wait(p_full + b, (j >> 1) & 1, abort_flag, status)) return false;
         tc::tc_fence_after();
         const uint32_t pcol = tmem + kColS + (uint32_t)(b * 128);
         const uint32_t ocol = tmem + kColO + (uint32_t)(b * D);  // O[b]: the stages of softmax group b
         for (int p = 0; p < np; ++p) {
-          const uint64_t vd = vd0 + (uint64_t)((u0 + p) % kSlots) * kStageStep;
+          const uint64_t vd = vd0 + (uint64_t)((u0 + p) % kVSlots) * kStageStep;
 #pragma unroll
           for (int k = 0; k < BN / 16; ++k)
             tc::mma_ts(ocol, pcol + (uint32_t)k * 8u, vd + (uint64_t)k * (2u * kGroup >> 4), id_o,
                        (j > 1 || p > 0 || k > 0) ? 1u : 0u);
         }
         tc::mma_commit(o_done + b);
-        for (int p = 0; p < np; ++p) tc::mma_commit(v_empty + (u0 + p) % kSlots);
+        for (int p = 0; p < np; ++p) tc::mma_commit(v_empty + (u0 + p) % kVSlots);
         return true;
       };
       for (int j = 0; ok && j < ntile; ++j) {
         const int b = j & 1, u0 = ustart(j), np = nparts(j);
         for (int p = 0; ok && p < np; ++p)
-          ok = tc::mbar_wait(k_full + (u0 + p) % kSlots, ((u0 + p) / kSlots) & 1, abort_flag, status);
+          ok = tc::mbar_wait(k_full + (u0 + p) % kKSlots, ((u0 + p) / kKSlots) & 1, abort_flag, status);
         if (!ok) break;
         tc::tc_fence_after();
         // S[b] was last read as P[b] by P.V of tile j-2, issued before
         const uint32_t scol = tmem + kColS + (uint32_t)(b * 128);
         for (int p = 0; p < np; ++p) {
-          const uint64_t kd = kd0 + (uint64_t)((u0 + p) % kSlots) * kStageStep;
+          const uint64_t kd = kd0 + (uint64_t)((u0 + p) % kKSlots) * kStageStep;
 #pragma unroll
           for (int k = 0; k < D / 16; ++k)
             tc::mma_ss(scol, qd + (uint64_t)((k >> 2) * 1024 + (k & 3) * 2), kd + (uint64_t)k * 16u, id_s,
                        (p > 0 || k > 0) ? 1u : 0u);
         }
         tc::mma_commit(s_full + b);
-        for (int p = 0; p < np; ++p) tc::mma_commit(k_empty + (u0 + p) % kSlots);
+        for (int p = 0; p < np; ++p) tc::mma_commit(k_empty + (u0 + p) % kKSlots);
         if (j > 0 && !issue_pv(j - 1)) { ok = false; break; }
       }
       if (ok && ntile > 0) issue_pv(ntile - 1);
@@ -418,11 +422,80 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc::mbar_arrive(q_full);
     }
     asm volatile("bar.sync 2, 96;" ::: "memory");  // range prefix ready
-    {
-      // one producer warp per ring slot (warp 1: even stages, warp 2: odd
-      // stages; warp 3 only helps with the query tile), so that the waits on a
-      // slot's barriers come in order and never run a phase ahead: keys once
-      // the K slot is free, values, bias and mask once the V slot is
+    // Pieces of the padded routed stream in [pos0, pos0 + BN): one lane per
+    // staged range from the first one that ends after pos0 (a routed range
+    // holds at least 8 padded rows, so the window meets at most 16 of them).
+    // A piece that would leave the stage tile or the packed rows gets zero
+    // groups (status word) and is neither copied nor unmasked.  Returns the
+    // piece count; tail = rows of the window the stream covers.
+    auto make_pieces = [&](int pos0, int4* pcs, int& tail, uint32_t& bytes) -> int {
+      const int end = pos0 + BN;
+      int npc = 0;
+      if (ns <= kMaxRanges) {
+        int ri = ns;
+        for (int base = 0; base < ns; base += 32) {
+          const int i = base + lane;
+          const unsigned m = __ballot_sync(0xffffffffu, i < ns && rng_cum[i + 1] > pos0);
+          if (m) { ri = base + __ffs(m) - 1; break; }
+        }
+        const int ci = ri + lane;
+        int lo = 0, hi = 0, cs = 0;
+        if (ci < ns) {
+          cs = rng_cum[ci];
+          lo = max(cs, pos0);
+          hi = min(rng_cum[ci + 1], end);
+        }
+        const bool has = hi > lo;
+        const unsigned hm = __ballot_sync(0xffffffffu, has);
+        int z = 0;
+        if (has) {
+          const int off = lo - cs;
+          int4 pc = make_int4((lo - pos0) >> 3, rng_start[ci] + off, (hi - lo) >> 3,
+                              max(0, min(rng_len[ci] - off, hi - lo)));
+          const bool good = pc.x >= 0 && pc.z > 0 && pc.x + pc.z <= BN / 8 && pc.y >= 0 &&
+                            (size_t)pc.y + (size_t)pc.z * 8 <= npad;
+          if (!good) { set_status(status, ST_BOUNDS); pc.z = 0; pc.w = 0; }
+          z = pc.z;
+          pcs[__popc(hm & ((1u << lane) - 1u))] = pc;
+        }
+        npc = __popc(hm);
+        tail = __reduce_max_sync(0xffffffffu, has ? hi - pos0 : 0);
+        // the window must be covered up to the stream end (status word if not)
+        if (lane == 0 && (long long)tail < min((long long)BN, lex - pos0)) set_status(status, ST_BOUNDS);
+        bytes = (uint32_t)__reduce_add_sync(0xffffffffu, z) * kGroup;
+      } else {
+        // more routed clusters than staged ranges: walk the selection list
+        int t = 0, nb = 0;
+        if (lane == 0) {
+          int cum = 0, pos = pos0;
+          for (int ri = 0; pos < end && ri < ns && npc < kMaxPieces; ++ri) {
+            const int c = sl[ri];
+            const int pst = pof[c], len = koff[c + 1] - koff[c], plen = (len + 7) & ~7;
+            if (cum + plen <= pos) { cum += plen; continue; }
+            const int off = pos - cum, take = min(plen - off, end - pos);
+            int4 pc = make_int4((pos - pos0) >> 3, pst + off, take >> 3, max(0, min(len - off, take)));
+            const bool good = pc.x >= 0 && pc.z > 0 && pc.x + pc.z <= BN / 8 && pc.y >= 0 &&
+                              (size_t)pc.y + (size_t)pc.z * 8 <= npad;
+            if (!good) { set_status(status, ST_BOUNDS); pc.z = 0; pc.w = 0; }
+            nb += pc.z;
+            pcs[npc++] = pc;
+            pos += take;
+            cum += plen;
+          }
+          t = pos - pos0;
+        }
+        npc = __shfl_sync(0xffffffffu, npc, 0);
+        tail = __shfl_sync(0xffffffffu, t, 0);
+        bytes = (uint32_t)__shfl_sync(0xffffffffu, nb, 0) * kGroup;
+      }
+      __syncwarp();
+      return npc;
+    };
+    // one producer warp per ring slot (warp 1: even stages, warp 2: odd
+    // stages; warp 3 only helps with the query tile), so that the waits on a
+    // slot's barriers come in order and never run a phase ahead: keys once
+    // the K slot is free, then values, bias and mask once the V slot is
+    if (warp == 1 || warp == 2) {
       const int pw = warp - 1;
       int4* pcs = pieces + pw * kMaxPieces;  // this warp's piece list
       const uint8_t* Kh = kpk + (size_t)h * npad * D * 2;
@@ -431,7 +504,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const size_t cbase = (size_t)h * Ckpad * D * 2;
       const int nstage = ustart(ntile);  // total ring stages of the stream
       const unsigned rot = n_ex > 0 ? (blockIdx.x * 2654435761u + h * 40503u) % (unsigned)n_ex : 0u;
-      for (int u = pw; pw < kSlots && u < nstage; u += kSlots) {
+      for (int u = pw; u < nstage; u += kSlots) {
         const int st = u % kSlots;
         const bool exact = u < n_ex;
         int j = exact ? u : n_ex + (u - n_ex) / 2;
@@ -440,81 +513,36 @@ __global__ void __launch_bounds__(kThreads, 1)
         // softmax does not depend on the order), so that the blocks of a head
         // do not all read the same popular clusters at the same time
         if (exact) j = (int)(((unsigned)j + rot) % (unsigned)n_ex);
-        const uint32_t ka = tc::smem_u32(smem + S::k_off + st * S::kKTile);
-        const uint32_t va = tc::smem_u32(smem + S::v_off + st * S::kKTile);
+        uint8_t* ktile = smem + S::k_off + st * S::kKTile;
+        uint8_t* vtile = smem + S::v_off + st * S::kKTile;
         int npc = 0, tail = BN;
-        uint32_t okm = 0, bytes = 0;
+        uint32_t bytes = 0;
         // ---- keys
         if (!tc::mbar_wait_warp(k_empty + st, ((u / kSlots) & 1) ^ 1, abort_flag, status)) break;
         if (exact) {
-          // pieces of the padded routed stream in [j*BN, j*BN + BN)
-          if (lane == 0) {
-            const int pos0 = j * BN, end = pos0 + BN;
-            int ri;
-            if (ns <= kMaxRanges) {
-              int lo = 0, hi = ns;  // largest i with cum[i] <= pos0
-              while (hi - lo > 1) {
-                const int mid = (lo + hi) >> 1;
-                if (rng_cum[mid] <= pos0) lo = mid; else hi = mid;
-              }
-              ri = lo;
-            } else {
-              ri = 0;
-            }
-            int cum = ns <= kMaxRanges ? rng_cum[ri] : 0;
-            int pos = pos0;
-            while (pos < end && ri < ns && npc < kMaxPieces) {
-              int pst, len;
-              if (ri < kMaxRanges) {
-                pst = rng_start[ri]; len = rng_len[ri];
-              } else {
-                const int c = sl[ri];
-                pst = pof[c]; len = koff[c + 1] - koff[c];
-              }
-              const int plen = (len + 7) & ~7;
-              if (cum + plen <= pos) { cum += plen; ++ri; continue; }  // (ranges past the staged prefix)
-              const int off = pos - cum, take = min(plen - off, end - pos);
-              pcs[npc++] = make_int4((pos - pos0) >> 3, pst + off, take >> 3, max(0, min(len - off, take)));
-              pos += take;
-              cum += plen;
-              ++ri;
-            }
-            tail = pos - pos0;
-            // a piece must stay inside the stage tile and the packed rows;
-            // one that does not is dropped (status word) instead of copied
-            for (int q = 0; q < npc; ++q) {
-              const int4 pc = pcs[q];
-              const bool good = pc.x >= 0 && pc.z > 0 && pc.x + pc.z <= BN / 8 && pc.y >= 0 &&
-                                (size_t)pc.y + (size_t)pc.z * 8 <= npad;
-              if (good) { okm |= 1u << q; bytes += (uint32_t)pc.z * kGroup; }
-              else set_status(status, ST_BOUNDS);
-            }
-          }
-          npc = __shfl_sync(0xffffffffu, npc, 0);
-          tail = __shfl_sync(0xffffffffu, tail, 0);
-          __syncwarp();
-          // zero the key rows past the stream end so the MMAs see finite values
+          npc = make_pieces(j * BN, pcs, tail, bytes);
+          // zero the rows past the stream end so the MMAs see finite values
           if (tail < BN) {
-            uint4* kz = reinterpret_cast<uint4*>(smem + S::k_off + st * S::kKTile) + (tail >> 3) * (kGroup / 16);
+            uint4* zr = reinterpret_cast<uint4*>(ktile) + (tail >> 3) * (kGroup / 16);
             const int nz = ((BN - tail) >> 3) * (int)(kGroup / 16);
-            for (int i = lane; i < nz; i += 32) kz[i] = make_uint4(0, 0, 0, 0);
+            for (int i = lane; i < nz; i += 32) zr[i] = make_uint4(0, 0, 0, 0);
             tc::fence_proxy_async();
           }
           __syncwarp();
           if (lane == 0) {
             tc::mbar_arrive_expect_tx(k_full + st, bytes);
             for (int q = 0; q < npc; ++q) {
-              if (!((okm >> q) & 1u)) continue;
               const int4 pc = pcs[q];
-              tc::bulk_g2s(ka + (uint32_t)pc.x * kGroup, Kh + (size_t)(pc.y >> 3) * kGroup,
-                           (uint32_t)pc.z * kGroup, k_full + st);
+              if (pc.z > 0)
+                tc::bulk_g2s(tc::smem_u32(ktile) + (uint32_t)pc.x * kGroup, Kh + (size_t)(pc.y >> 3) * kGroup,
+                             (uint32_t)pc.z * kGroup, k_full + st);
             }
           }
         } else if (lane == 0) {
           const uint32_t n = (uint32_t)(BN / 8) * kGroup;
           const size_t go = cbase + (size_t)(((j - n_ex) * BN) >> 3) * kGroup;
           tc::mbar_arrive_expect_tx(k_full + st, n);
-          tc::bulk_g2s(ka, (p == 0 ? kb_hi : kb_lo) + go, n, k_full + st);
+          tc::bulk_g2s(tc::smem_u32(ktile), (p == 0 ? kb_hi : kb_lo) + go, n, k_full + st);
         }
         __syncwarp();
         // ---- values, bias and mask
@@ -529,9 +557,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int i = lane; i < pc.w; i += 32) bias[pc.x * 8 + i] = 0.f;
           }
           if (tail < BN) {
-            uint4* vz = reinterpret_cast<uint4*>(smem + S::v_off + st * S::kKTile) + (tail >> 3) * (kGroup / 16);
+            uint4* zr = reinterpret_cast<uint4*>(vtile) + (tail >> 3) * (kGroup / 16);
             const int nz = ((BN - tail) >> 3) * (int)(kGroup / 16);
-            for (int i = lane; i < nz; i += 32) vz[i] = make_uint4(0, 0, 0, 0);
+            for (int i = lane; i < nz; i += 32) zr[i] = make_uint4(0, 0, 0, 0);
             tc::fence_proxy_async();
           }
           if (lane == 0) flag_s[st] = 1;
@@ -539,10 +567,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (lane == 0) {
             tc::mbar_arrive_expect_tx(v_full + st, bytes);
             for (int q = 0; q < npc; ++q) {
-              if (!((okm >> q) & 1u)) continue;
               const int4 pc = pcs[q];
-              tc::bulk_g2s(va + (uint32_t)pc.x * kGroup, Vh + (size_t)(pc.y >> 3) * kGroup,
-                           (uint32_t)pc.z * kGroup, v_full + st);
+              if (pc.z > 0)
+                tc::bulk_g2s(tc::smem_u32(vtile) + (uint32_t)pc.x * kGroup, Vh + (size_t)(pc.y >> 3) * kGroup,
+                             (uint32_t)pc.z * kGroup, v_full + st);
             }
           }
         } else {
@@ -560,7 +588,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint32_t n = (uint32_t)(BN / 8) * kGroup;
             const size_t go = cbase + (size_t)(c0 >> 3) * kGroup;
             tc::mbar_arrive_expect_tx(v_full + st, n);
-            tc::bulk_g2s(va, (p == 0 ? vb_hi : vb_lo) + go, n, v_full + st);
+            tc::bulk_g2s(tc::smem_u32(vtile), (p == 0 ? vb_hi : vb_lo) + go, n, v_full + st);
           }
         }
         __syncwarp();
@@ -579,11 +607,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     float m_used = -INFINITY, l = 0.f;
     bool ok = true;
     for (int j = w; ok && j < ntile; j += 2) {
-      const int u0 = ustart(j), st = u0 % kSlots;
+      const int u0 = ustart(j), st = u0 % kVSlots;
       if (!tc::mbar_wait_warp(s_full + w, (j >> 1) & 1, abort_flag, status)) { ok = false; break; }
       // bias / mask of this stage: acquire the producers' writes through the
       // stage's V barrier (its next phase needs this stage's P.V first)
-      if (!tc::mbar_wait_warp(v_full + st, (u0 / kSlots) & 1, abort_flag, status)) { ok = false; break; }
+      if (!tc::mbar_wait_warp(v_full + st, (u0 / kVSlots) & 1, abort_flag, status)) { ok = false; break; }
       tc::tc_fence_after();
       const float* bias = bias_s + st * BN;
       // pass 1: the row maximum over the stage's 128 keys, 64 at a time
