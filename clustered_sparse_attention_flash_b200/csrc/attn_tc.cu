@@ -54,9 +54,8 @@ constexpr int BQ = 128;        // rows per query tile (one tile per block)
 constexpr int BN = 128;        // keys per ring stage
 constexpr int kThreads = 384;
 constexpr int kProducers = 96;
-constexpr int kSlots = 2;      // K ring and V ring
-constexpr int kKSlots = kSlots;
-constexpr int kVSlots = kSlots;
+constexpr int kKSlots = 3;     // K ring (keys are needed first)
+constexpr int kVSlots = 2;     // V ring (with the stage's bias vector)
 constexpr int kUnitRows = BQ;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr uint32_t kColS = 0, kColO = 256;
@@ -491,10 +490,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       __syncwarp();
       return npc;
     };
-    // one producer warp per ring slot (warp 1: even stages, warp 2: odd
-    // stages; warp 3 only helps with the query tile), so that the waits on a
-    // slot's barriers come in order and never run a phase ahead: keys once
-    // the K slot is free, then values, bias and mask once the V slot is
+    // warp 1 produces the even stages, warp 2 the odd ones (warp 3 only helps
+    // with the query tile): keys once the K slot is free, then values, bias
+    // and mask once the V slot is.  A warp reaches stage u only after its
+    // stage u - 2 saw P.V of stage u - 4 complete, so every S and P.V up to
+    // there is done and no wait on a ring barrier can run a phase ahead.
     if (warp == 1 || warp == 2) {
       const int pw = warp - 1;
       int4* pcs = pieces + pw * kMaxPieces;  // this warp's piece list
@@ -504,8 +504,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       const size_t cbase = (size_t)h * Ckpad * D * 2;
       const int nstage = ustart(ntile);  // total ring stages of the stream
       const unsigned rot = n_ex > 0 ? (blockIdx.x * 2654435761u + h * 40503u) % (unsigned)n_ex : 0u;
-      for (int u = pw; u < nstage; u += kSlots) {
-        const int st = u % kSlots;
+      for (int u = pw; u < nstage; u += 2) {
+        const int sk = u % kKSlots, st = u % kVSlots;
         const bool exact = u < n_ex;
         int j = exact ? u : n_ex + (u - n_ex) / 2;
         const int p = exact ? 0 : (u - n_ex) & 1;
@@ -513,12 +513,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         // softmax does not depend on the order), so that the blocks of a head
         // do not all read the same popular clusters at the same time
         if (exact) j = (int)(((unsigned)j + rot) % (unsigned)n_ex);
-        uint8_t* ktile = smem + S::k_off + st * S::kKTile;
+        uint8_t* ktile = smem + S::k_off + sk * S::kKTile;
         uint8_t* vtile = smem + S::v_off + st * S::kKTile;
         int npc = 0, tail = BN;
         uint32_t bytes = 0;
         // ---- keys
-        if (!tc::mbar_wait_warp(k_empty + st, ((u / kSlots) & 1) ^ 1, abort_flag, status)) break;
+        if (!tc::mbar_wait_warp(k_empty + sk, ((u / kKSlots) & 1) ^ 1, abort_flag, status)) break;
         if (exact) {
           npc = make_pieces(j * BN, pcs, tail, bytes);
           // zero the rows past the stream end so the MMAs see finite values
@@ -530,23 +530,23 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           __syncwarp();
           if (lane == 0) {
-            tc::mbar_arrive_expect_tx(k_full + st, bytes);
+            tc::mbar_arrive_expect_tx(k_full + sk, bytes);
             for (int q = 0; q < npc; ++q) {
               const int4 pc = pcs[q];
               if (pc.z > 0)
                 tc::bulk_g2s(tc::smem_u32(ktile) + (uint32_t)pc.x * kGroup, Kh + (size_t)(pc.y >> 3) * kGroup,
-                             (uint32_t)pc.z * kGroup, k_full + st);
+                             (uint32_t)pc.z * kGroup, k_full + sk);
             }
           }
         } else if (lane == 0) {
           const uint32_t n = (uint32_t)(BN / 8) * kGroup;
           const size_t go = cbase + (size_t)(((j - n_ex) * BN) >> 3) * kGroup;
-          tc::mbar_arrive_expect_tx(k_full + st, n);
-          tc::bulk_g2s(tc::smem_u32(ktile), (p == 0 ? kb_hi : kb_lo) + go, n, k_full + st);
+          tc::mbar_arrive_expect_tx(k_full + sk, n);
+          tc::bulk_g2s(tc::smem_u32(ktile), (p == 0 ? kb_hi : kb_lo) + go, n, k_full + sk);
         }
         __syncwarp();
         // ---- values, bias and mask
-        if (!tc::mbar_wait_warp(v_empty + st, ((u / kSlots) & 1) ^ 1, abort_flag, status)) break;
+        if (!tc::mbar_wait_warp(v_empty + st, ((u / kVSlots) & 1) ^ 1, abort_flag, status)) break;
         float* bias = bias_s + st * BN;
         if (exact) {
           // bias: valid keys 0, padding and the stream tail -inf
