@@ -144,11 +144,11 @@ def _peaks():
 
 # DRAM traffic of the attention kernel from one ncu capture (dram__bytes_read.sum
 # + dram__bytes_write.sum of k_attn_tc on the first 4 heads of the Wan-shaped
-# workload: 345.5 MB, i.e. 86.4 MB per head; traffic grows with the heads).  The
+# workload: 324.9 MB, i.e. 81.2 MB per head; traffic grows with the heads).  The
 # figure holds only for the kernel sources it was taken on, identified by hash.
-_ATTN_TRAFFIC = {"bytes_per_head": 345.5e6 / 4, "workload": "wan",
+_ATTN_TRAFFIC = {"bytes_per_head": 324.9e6 / 4, "workload": "wan",
                  "sources": ("attn_tc.cu", "attn_tc.cuh", "tc_common.cuh"),
-                 "sha1": "5fdd31828da8cb2c8124a5982d6717bc21d423de"}
+                 "sha1": "f7e1b11454368752bc9b16368575da9f2ea41927"}
 
 
 def attn_traffic(cfg):

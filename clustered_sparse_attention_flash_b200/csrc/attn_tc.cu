@@ -19,26 +19,27 @@
 // padded to a multiple of 8 rows, each group of 8 rows stored as
 // [16-byte chunk][row]), which is directly a no-swizzle UMMA operand (K-major
 // for K, MN-major for V); a stage is one or a few contiguous runs, each moved
-// by a single cp.async.bulk.  K and V have separate two-slot rings: a K slot is
-// free once S of its tile is computed, a V slot (and the stage's bias vector)
-// once P.V is; padding rows are masked through the bias vector.
+// by a single cp.async.bulk.  K has a three-slot ring and V (with the stage's
+// bias vector) a two-slot ring: a K slot is free once S of its stage is
+// computed, a V slot once P.V is; padding rows are masked through the bias.
 // Warp roles (12 warps):
 //   warp 0      tensor-memory allocation, MMA issue (one thread): S = Q K^T
-//               into double-buffered S (N = 128 keys), then O += P V of the
-//               previous tile with P read from tensor memory;
+//               into double-buffered S (N = 128 keys), then O[j % 2] += P V of
+//               the previous stage with P read from tensor memory;
 //   warps 1-3   load the query tile; warps 1 and 2 then produce the even
 //               and the odd stages (bulk copies issued by one lane, bias
 //               vectors by the warp);
-//   warps 4-7   softmax of keys 0..63 of every stage, warps 8-11 of keys
-//               64..127 (thread = query row): the two halves exchange their
-//               row maxima through shared memory, rescale O lazily (each its
-//               half of the d columns) when the maximum grows by more than 2^8,
-//               write P = 2^(x - m) in bf16 over the S columns of the stage
-//               and finally store O / l through perm_q.
-// Tensor memory (512 columns): S[0..1] [0,256), O [256,256+d); P[b] lives in
-// the first 64 columns of S[b].  Every decision that guards a warp-collective
-// tensor-memory access is made warp-uniform, and every wait is time-bounded
-// (device status word on expiry).
+//   warps 4-7   softmax of the even stages, warps 8-11 of the odd stages
+//               (thread = query row, all 128 keys of its stage): each group
+//               keeps its own running maximum, row sum and accumulator O[w],
+//               rescales O[w] lazily when its maximum grows by more than 2^8,
+//               writes P = 2^(x - m) in bf16 over the S columns of the stage;
+//               at the end the two partial results are merged (split-K style)
+//               and O / l is stored through perm_q.
+// Tensor memory (512 columns): S[0..1] [0,256), O[0..1] [256,256+2d); P[b]
+// lives in the first 64 columns of S[b].  Every decision that guards a
+// warp-collective tensor-memory access is made warp-uniform, and every wait
+// is time-bounded (device status word on expiry).
 #include <algorithm>
 #include <cmath>
 
