@@ -225,6 +225,23 @@ def dense_flops(cfg):
     return 4.0 * cfg.H * cfg.N * cfg.N * cfg.d
 
 
+def max_over_ranks(x, dist=None, device="cpu"):
+    """The largest x over all ranks (the slowest rank's time); x itself with
+    one process."""
+    if dist is None:
+        return float(x)
+    import torch
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_value(cfg, world, ms):
+    """Whole-job dense-equivalent TFLOP/s: every rank runs one full layer of
+    cfg (weak scaling), timed by the slowest rank's ms per layer."""
+    return world * dense_flops(cfg) / (ms / 1e3) / 1e12
+
+
 def run_reference(a, cfg, rho):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
@@ -324,11 +341,7 @@ def main():
         torch.cuda.synchronize(dev)
     launches = sv.svgear_launch_count() - l0
     barrier()
-    ms = ev0.elapsed_time(ev1) / a.steps
-    if dist is not None:
-        t = torch.tensor([ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = max_over_ranks(ev0.elapsed_time(ev1) / a.steps, dist, dev)
     clocks = clk.summary()
 
     # ---- per-stage breakdown (library-internal CUDA events on the same stream)
@@ -357,14 +370,10 @@ def main():
             hO.copy_(dO, non_blocking=True)
         e1.record(stream)
         torch.cuda.synchronize(dev)
-        ems = e0.elapsed_time(e1) / a.steps
-        if dist is not None:
-            t = torch.tensor([ems], device=dev)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            ems = float(t.item())
+        ems = max_over_ranks(e0.elapsed_time(e1) / a.steps, dist, dev)
         bi = 3 * Q.numel() * Q.element_size()
         bo = hO.numel() * hO.element_size()
-        e2e = {"value": world * dense_flops(cfg) / (ems / 1e3) / 1e12, "unit": UNIT,
+        e2e = {"value": job_value(cfg, world, ems), "unit": UNIT,
                "h2d_bytes_per_step": bi, "d2h_bytes_per_step": bo, "ms_per_step": ems}
 
     peak_tc, peak_hbm, peak_src = _peaks()
@@ -383,7 +392,7 @@ def main():
         cpu = {"value": dense_flops(cfg) / sec / 1e12, "unit": UNIT, "cores": _threads(),
                "kind": "oracle", "sample": desc, "layer_s_extrapolated": sec}
 
-    value = world * dense_flops(cfg) / (ms / 1e3) / 1e12
+    value = job_value(cfg, world, ms)
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": a.steps,
         "warmup": a.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",

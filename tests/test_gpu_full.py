@@ -1,0 +1,75 @@
+"""Parity at the full Wan-shaped size, in the launch configuration bench.py
+times: all 40 heads (N = 75,600, d = 128, Cq = 100, Ck = 500, rho = 0.15, ten
+k-means rounds) in one svgear_forward.  The oracle cannot run the whole layer,
+so on sampled heads and rows every stage is checked against the oracle given
+the GPU's own inputs to that stage."""
+import math
+
+import numpy as np
+import pytest
+
+from clustered_sparse_attention_flash_b200 import svgear as sv
+from clustered_sparse_attention_flash_b200 import synth
+from oracle import svgear_oracle as ora
+
+from helpers import E_FLOOR, E_RTOL, OUT_TOL, TIE_REL, assert_close, dev, host, label_mismatches_are_ties
+
+
+def _tied_rows(Erow, kc):
+    order = ora.route_order(Erow, kc)
+    v = Erow[order]
+    return (np.abs(np.diff(v)) <= TIE_REL * np.maximum(np.abs(v[:-1]), 1e-300)).any()
+
+
+@pytest.mark.gpu
+def test_wan_layer_sampled_parity():
+    import torch
+    import bench
+    cfg = synth.CONFIGS["wan"]
+    q, k, v, iq, ik = bench.generate(cfg)
+    s = 1.0 / math.sqrt(cfg.d)
+    bf = torch.bfloat16
+    O, ws, p, _ = sv.forward(dev(q, bf), dev(k, bf), dev(v, bf), cfg.Cq, cfg.Ck, cfg.iters, cfg.rho, s,
+                             dev(iq), dev(ik))
+    torch.cuda.synchronize()
+    assert sv.svgear_get_status() == sv.SVGEAR_OK
+    vw = sv.view_tensors(p, ws)
+    rng = np.random.default_rng(20260)
+    for h in (0, 27):
+        Q, K, V = q[h], k[h], v[h]
+        cq, ck, vbar = (host(vw[n][h]).astype(np.float64) for n in ("cent_q", "cent_k", "vbar"))
+        lq, lk = host(vw["labels_q"][h]), host(vw["labels_k"][h])
+        # a1: labels are the exact argmin for the final centroids (ties exempt)
+        label_mismatches_are_ties(Q, cq, lq)
+        label_mismatches_are_ties(K, ck, lk)
+        # a3: counts, offsets and the stable permutation follow the labels;
+        # value centroids are the member means
+        cnt_k = host(vw["counts_k"][h])
+        assert np.array_equal(cnt_k, np.bincount(lk, minlength=cfg.Ck))
+        assert np.array_equal(host(vw["off_k"][h]), np.concatenate([[0], np.cumsum(cnt_k)]))
+        assert np.array_equal(host(vw["perm_k"][h]), np.argsort(lk, kind="stable"))
+        assert np.array_equal(host(vw["counts_q"][h]), np.bincount(lq, minlength=cfg.Cq))
+        assert_close(vbar, ora.value_centroids(V, lk, cfg.Ck), 1e-5, 1e-5, "value centroids")
+        # a4: block error from these clusters
+        args = (cq, ck, vbar, K, V, lk, cnt_k, s)
+        Eo, Mo = ora.block_error(*args)
+        T = ora.block_error_scale(*args)
+        E = host(vw["E"][h])
+        assert_close(host(vw["M"][h]), Mo, 1e-5, 1e-6, "row shift M")
+        err = np.abs(E - Eo)
+        lim = E_RTOL * np.abs(Eo) + E_FLOOR * T
+        assert (err <= lim).all(), f"E: {(err > lim).sum()} entries outside"
+        # a5: routing from the GPU's errors (rows with near-tied ratios exempt)
+        cnt_q = host(vw["counts_q"][h])
+        mask_o, _, _ = ora.route(E, cnt_k, cnt_q, cfg.rho)
+        mask = host(vw["mask"][h])
+        for a in range(cfg.Cq):
+            if not np.array_equal(mask[a], mask_o[a]):
+                assert _tied_rows(E[a], cnt_k), f"routing row {a} differs without a tie"
+        # a6: 256 sampled query rows against the oracle's hybrid attention
+        rows = rng.choice(cfg.N, 256, replace=False)
+        lq_s = np.full_like(lq, -1)
+        lq_s[rows] = lq[rows]
+        Oo = ora.hybrid_attention(Q, K, V, lq_s, lk, ck, vbar, cnt_k, mask, s)
+        atol, rtol = OUT_TOL["bf16"]
+        assert_close(host(O[h])[rows], Oo[rows], atol, rtol, f"hybrid output head {h}")
