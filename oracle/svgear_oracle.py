@@ -235,6 +235,70 @@ def block_error_scale(Qbar, Kbar, Vbar, K, V, k_labels, k_counts, scale: float,
 
 
 # --------------------------------------------------------------------------
+# (2') routing-signal ablations.  The pages contrast error-aware routing with
+#      selectors that rank blocks by attention score ([AB]; [DE] 2.B; [IT]
+#      2.B): these two swap the ranking signal and keep every other step.
+# --------------------------------------------------------------------------
+
+def block_mass(Qbar, Kbar, k_counts, scale: float):
+    """Score-based signal: the attention weight the query centroid qbar_a
+    gives key cluster c when every key of c is replaced by kbar_c,
+
+        P[a, c] = |k_c| exp(s qbar_a.kbar_c) / sum_{c' non-empty} |k_c'| exp(s qbar_a.kbar_c'),
+
+    0 for empty clusters; each row sums to 1.  Returns (P [Cq, Ck], M [Cq])
+    with M as in block_error."""
+    k_counts = np.asarray(k_counts)
+    M = block_shift(Qbar, Kbar, k_counts, scale)
+    L = scale * (_f64(Qbar) @ _f64(Kbar).T)
+    nz = k_counts > 0
+    P = np.zeros_like(L)
+    P[:, nz] = k_counts[nz][None, :] * np.exp(L[:, nz] - M[:, None])
+    P /= P.sum(axis=1, keepdims=True)
+    return P, M
+
+
+def block_error_value_agnostic(Qbar, Kbar, K, k_labels, k_counts, scale: float,
+                               key_chunk: int = 1024):
+    """The block error with the values left out:
+
+        eps^2(a, j) = (exp(s qbar_a.kbar_c) - exp(s qbar_a.k_j))^2
+        E[a, c]     = exp(-2 M_a) * (1/|k_c|) * sum_{j in c} eps^2(a, j)
+
+    Returns (E [Cq, Ck], M [Cq]); empty key clusters get 0."""
+    Qbar, Kbar, K = map(_f64, (Qbar, Kbar, K))
+    k_labels = np.asarray(k_labels)
+    k_counts = np.asarray(k_counts)
+    M = block_shift(Qbar, Kbar, k_counts, scale)
+    Lbar = scale * (Qbar @ Kbar.T)
+    E = np.zeros((Qbar.shape[0], Kbar.shape[0]))
+    for s in range(0, K.shape[0], key_chunk):
+        j = slice(s, s + key_chunk)
+        c = k_labels[j]
+        A = np.exp(Lbar[:, c] - M[:, None])
+        B = np.exp(scale * (Qbar @ K[j].T) - M[:, None])
+        np.add.at(E.T, c, ((A - B) ** 2).T)
+    nz = k_counts > 0
+    E[:, nz] /= k_counts[nz][None, :]
+    return E, M
+
+
+ROUTERS = ("error", "mass", "error_nov")
+
+
+def routing_signal(router: str, Qbar, Kbar, Vbar, K, V, k_labels, k_counts, scale: float):
+    """(E, M) for the named signal: "error" (the method), "mass" or
+    "error_nov" (the ablations above)."""
+    if router == "error":
+        return block_error(Qbar, Kbar, Vbar, K, V, k_labels, k_counts, scale)
+    if router == "mass":
+        return block_mass(Qbar, Kbar, k_counts, scale)
+    if router == "error_nov":
+        return block_error_value_agnostic(Qbar, Kbar, K, k_labels, k_counts, scale)
+    raise ValueError(router)
+
+
+# --------------------------------------------------------------------------
 # (3) error-aware routing under the density budget rho
 #     [R] step (3); [DE] 2.B "Selektion"; [IT] 2.B "Selezione Greedy"
 # --------------------------------------------------------------------------
@@ -328,14 +392,15 @@ def dense_attention(Q, K, V, scale: float) -> np.ndarray:
 # --------------------------------------------------------------------------
 
 def forward(Q, K, V, Cq: int, Ck: int, iters: int, rho, scale: float,
-            init_q, init_k) -> Dict[str, object]:
-    """All steps of one head in order; returns every intermediate."""
+            init_q, init_k, router: str = "error") -> Dict[str, object]:
+    """All steps of one head in order; returns every intermediate.  `router`
+    names the routing signal (ROUTERS; "error" is the method)."""
     Qbar, lq, cq = kmeans(Q, Cq, iters, init_q)
     Kbar, lk, ck = kmeans(K, Ck, iters, init_k)
     perm_q, off_q, _ = permute(lq, Cq)
     perm_k, off_k, _ = permute(lk, Ck)
     Vbar = value_centroids(V, lk, Ck)
-    E, M = block_error(Qbar, Kbar, Vbar, K, V, lk, ck, scale)
+    E, M = routing_signal(router, Qbar, Kbar, Vbar, K, V, lk, ck, scale)
     mask, sel, pairs = route(E, ck, cq, rho)
     O = hybrid_attention(Q, K, V, lq, lk, Kbar, Vbar, ck, mask, scale)
     return dict(Qbar=Qbar, Kbar=Kbar, Vbar=Vbar, q_labels=lq, k_labels=lk,

@@ -205,6 +205,76 @@ def test_block_error_equals_pairwise_ratio_bruteforce():
             assert E[a, c] == pytest.approx(want, rel=1e-11, abs=1e-300)
 
 
+# ------------------------------------------------------ routing ablations ----
+
+def test_block_mass_is_the_compensated_attention_weight():
+    """With every block compensated, hybrid attention of the query centroid
+    gives cluster c the weight |k_c| e^{s qbar.kbar_c} / sum; reading those
+    weights out through one-hot value centroids must give block_mass."""
+    rng = np.random.default_rng(21)
+    Nk, d, Cq, Ck, s = 50, 6, 3, 6, 0.8       # d = Ck: the one-hot values fit the output rows
+    K = rng.standard_normal((Nk, d))
+    lk = rng.integers(0, Ck - 1, Nk)            # cluster Ck-1 stays empty
+    ck = np.bincount(lk, minlength=Ck)
+    Kb = ora.value_centroids(K, lk, Ck)
+    Qb = rng.standard_normal((Cq, d))
+    P, M = ora.block_mass(Qb, Kb, ck, s)
+    O = ora.hybrid_attention(Qb, K, np.zeros((Nk, Ck)), np.arange(Cq), lk, Kb, np.eye(Ck), ck,
+                             np.zeros((Cq, Ck), np.uint8), s)
+    np.testing.assert_allclose(P, O, rtol=1e-12, atol=1e-15)
+    assert (P[:, -1] == 0).all()
+    np.testing.assert_allclose(P.sum(1), 1.0, rtol=1e-14)
+    np.testing.assert_allclose(M, ora.block_shift(Qb, Kb, ck, s))
+
+
+def test_block_mass_equal_logits_is_cluster_share():
+    """qbar = 0: every logit is 0, so the mass of c is |k_c| / N_k."""
+    ck = np.array([3, 0, 5, 2])
+    P, _ = ora.block_mass(np.zeros((2, 3)), np.ones((4, 3)), ck, 0.7)
+    np.testing.assert_allclose(P, np.broadcast_to(ck / ck.sum(), P.shape), rtol=1e-15)
+
+
+def test_value_agnostic_error_is_value_aware_with_constant_values():
+    """v_j = vbar_c = u with |u| = 1 turns eps^2 into (A - B_j)^2."""
+    rng = np.random.default_rng(22)
+    Nk, d, Cq, Ck, s = 40, 5, 4, 5, 0.6
+    K = rng.standard_normal((Nk, d))
+    lk = rng.integers(0, Ck, Nk)
+    ck = np.bincount(lk, minlength=Ck)
+    Kb = ora.value_centroids(K, lk, Ck)
+    Qb = rng.standard_normal((Cq, d))
+    u = rng.standard_normal(d); u /= np.linalg.norm(u)
+    Ev, Mv = ora.block_error(Qb, Kb, np.tile(u, (Ck, 1)), K, np.tile(u, (Nk, 1)), lk, ck, s)
+    En, Mn = ora.block_error_value_agnostic(Qb, Kb, K, lk, ck, s)
+    np.testing.assert_allclose(En, Ev, rtol=1e-12, atol=1e-300)
+    np.testing.assert_array_equal(Mn, Mv)
+
+
+def test_value_agnostic_two_key_closed_form():
+    """The two-key case of the value-aware pin without its values:
+    E = (1/2) ((1 - e^-1)^2 + (e - 1)^2)."""
+    E, M = ora.block_error_value_agnostic(np.array([[1.0]]), np.array([[1.0]]),
+                                          np.array([[0.0], [2.0]]), np.array([0, 0]), np.array([2]), 1.0)
+    e = math.e
+    assert M[0] == pytest.approx(1.0)
+    assert E[0, 0] == pytest.approx(0.5 * ((1 - 1 / e) ** 2 + (e - 1) ** 2), rel=1e-13)
+
+
+def test_routing_signal_dispatch():
+    rng = np.random.default_rng(23)
+    K = rng.standard_normal((30, 3)); V = rng.standard_normal((30, 3))
+    lk = rng.integers(0, 4, 30); ck = np.bincount(lk, minlength=4)
+    Kb = ora.value_centroids(K, lk, 4); Vb = ora.value_centroids(V, lk, 4)
+    Qb = rng.standard_normal((2, 3))
+    args = (Qb, Kb, Vb, K, V, lk, ck, 0.5)
+    np.testing.assert_array_equal(ora.routing_signal("error", *args)[0], ora.block_error(*args)[0])
+    np.testing.assert_array_equal(ora.routing_signal("mass", *args)[0], ora.block_mass(Qb, Kb, ck, 0.5)[0])
+    np.testing.assert_array_equal(ora.routing_signal("error_nov", *args)[0],
+                                  ora.block_error_value_agnostic(Qb, Kb, K, lk, ck, 0.5)[0])
+    with pytest.raises(ValueError):
+        ora.routing_signal("score", *args)
+
+
 # ----------------------------------------------------------------- routing ----
 
 def test_route_extremes_and_budget():
@@ -314,6 +384,15 @@ def test_hybrid_rho_zero_is_biased_centroid_attention():
     want = _sdpa64(Q, out["Kbar"][nz], out["Vbar"][nz], s,
                    bias=np.log(out["k_counts"][nz].astype(float))[None, :])
     np.testing.assert_allclose(out["O"], want, rtol=1e-10, atol=1e-12)
+
+
+@pytest.mark.parametrize("router", ["mass", "error_nov"])
+def test_ablation_routers_rho_one_is_dense(router):
+    """Whatever the ranking signal, rho = 1 routes every non-empty cluster."""
+    Q, K, V, Cq, Ck = _small_case(15)
+    s = 1 / math.sqrt(8)
+    out = ora.forward(Q, K, V, Cq, Ck, 3, 1.0, s, Q[:Cq], K[:Ck], router=router)
+    np.testing.assert_allclose(out["O"], _sdpa64(Q, K, V, s), rtol=1e-10, atol=1e-12)
 
 
 def test_forward_invariant_to_token_permutation():
