@@ -46,6 +46,9 @@ def _args():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--heads", type=int, default=None,
                     help="run only the first H heads of the workload (small profiler captures)")
+    ap.add_argument("--stress", action="store_true",
+                    help="error against dense attention over the noise sigma x budget rho grid "
+                         "of the stress workload, for the method's router and two ablations")
     return ap.parse_args()
 
 
@@ -57,9 +60,8 @@ def _workload(cfg, rho):
 
 
 def _gen_head(args):
-    name, h = args
+    cfg, h = args
     from clustered_sparse_attention_flash_b200 import synth
-    cfg = synth.CONFIGS[name]
     q, k, v, _ = synth.make_head(cfg, h)
     iq = synth.forgy_init(cfg, q, h, 0, cfg.Cq)
     ik = synth.forgy_init(cfg, k, h, 1, cfg.Ck)
@@ -75,9 +77,9 @@ def generate(cfg):
     n = min(8, os.cpu_count() or 1, cfg.H)
     if n > 1:
         with mp.get_context("spawn").Pool(n) as pool:
-            parts = pool.map(_gen_head, [(cfg.name, h) for h in range(cfg.H)])
+            parts = pool.map(_gen_head, [(cfg, h) for h in range(cfg.H)])
     else:
-        parts = [_gen_head((cfg.name, h)) for h in range(cfg.H)]
+        parts = [_gen_head((cfg, h)) for h in range(cfg.H)]
     return [np.stack([p[i] for p in parts]) for i in range(5)]
 
 
@@ -270,10 +272,103 @@ def run_reference(a, cfg, rho):
     return 0
 
 
+# ------------------------------------------------------------------ stress
+
+def _dense_fp32(Q, K, V, scale, rows=4096):
+    """softmax(s Q K^T) V per head in float32 (TF32 off), query rows chunked."""
+    import torch
+    O = torch.empty_like(Q)
+    for h in range(Q.shape[0]):
+        for r in range(0, Q.shape[1], rows):
+            S = torch.matmul(Q[h, r:r + rows], K[h].T) * scale
+            O[h, r:r + rows] = torch.matmul(torch.softmax(S, dim=-1), V[h])
+    return O
+
+
+def _nonincreasing(xs, slack=1.0):
+    return all(b <= a * slack for a, b in zip(xs, xs[1:]))
+
+
+def run_stress(a):
+    """Relative L2 and max error of the operator's output against dense
+    attention on the stress workload (H=16, N=32,768, d=128, Cq=64, Ck=512),
+    for each within-center noise sigma and density budget rho, with the
+    method's error-aware router and the two ablation signals.  The yardstick is
+    float32 dense attention on the GPU; rows of it are checked in float64."""
+    from clustered_sparse_attention_flash_b200 import synth
+    base = synth.CONFIGS["stress"]
+    if a.heads is not None:
+        base = base.with_(H=a.heads)
+    sigmas, rhos = synth.STRESS_SIGMAS, synth.STRESS_RHOS
+    data = {sg: generate(base.with_(sigma=sg)) for sg in sigmas}   # before any CUDA call
+
+    import numpy as np
+    import torch
+    from clustered_sparse_attention_flash_b200 import svgear as sv
+    torch.backends.cuda.matmul.allow_tf32 = False
+    torch.backends.cudnn.allow_tf32 = False
+    dev = torch.device("cuda", 0)
+    s = 1.0 / math.sqrt(base.d)
+    routers = (("error", sv.SVGEAR_ROUTE_ERROR), ("mass", sv.SVGEAR_ROUTE_MASS),
+               ("error_nov", sv.SVGEAR_ROUTE_ERROR_NOV))
+    rows = []
+    yard = {}
+    t0 = time.perf_counter()
+    for sg in sigmas:
+        q, k, v, iq, ik = data[sg]
+        dQ, dK, dV = (torch.from_numpy(x).to(dev).to(torch.bfloat16) for x in (q, k, v))
+        diq, dik = torch.from_numpy(iq).to(dev), torch.from_numpy(ik).to(dev)
+        Of = [x.float() for x in (dQ, dK, dV)]
+        ref = _dense_fp32(*Of, s)
+        # the yardstick against float64 on 256 rows of head 0
+        r64 = torch.softmax(torch.matmul(Of[0][0, :256].double(), Of[1][0].double().T) * s, dim=-1) @ Of[2][0].double()
+        yard[sg] = float((ref[0, :256].double() - r64).abs().max())
+        nref = float(torch.linalg.vector_norm(ref.double()))
+        ws = None
+        for rname, rcode in routers:
+            for rho in rhos:
+                O, ws, p, st = sv.forward(dQ, dK, dV, base.Cq, base.Ck, base.iters, rho, s, diq, dik,
+                                          ws=ws, stats=True, router=rcode)
+                if sv.svgear_get_status() != sv.SVGEAR_OK:
+                    raise RuntimeError("device status not OK")
+                d = O.float() - ref
+                rows.append({"sigma": sg, "rho": rho, "router": rname,
+                             "rel_l2": float(torch.linalg.vector_norm(d.double())) / nref,
+                             "max_abs": float(d.abs().max()),
+                             "density": st["exec_pairs"] / (base.H * base.N * base.N),
+                             "ms": st["ms_total"]})
+        del dQ, dK, dV, Of, ref
+        torch.cuda.empty_cache()
+
+    def err(sg, rho, r="error"):
+        return next(x["rel_l2"] for x in rows if x["sigma"] == sg and x["rho"] == rho and x["router"] == r)
+
+    trends = {
+        # error against dense must not fall as the noise grows (fixed rho) ...
+        "nondecreasing_in_sigma": {str(rho): _nonincreasing([err(sg, rho) for sg in sigmas][::-1])
+                                   for rho in rhos},
+        # ... and must not rise as the budget grows (fixed sigma)
+        "nonincreasing_in_rho": {str(sg): _nonincreasing([err(sg, rho) for rho in rhos]) for sg in sigmas},
+        "error_router_best": {f"{sg}/{rho}": min(("error", "mass", "error_nov"), key=lambda r: err(sg, rho, r))
+                              for sg in sigmas for rho in rhos},
+    }
+    line = {"stress": True, "workload": _workload(base, "swept"), "sigmas": sigmas, "rhos": rhos,
+            "yardstick": "float32 dense attention on the GPU (TF32 off) from the same bf16 inputs",
+            "yardstick_max_abs_vs_float64_256_rows": yard, "results": rows, "trends": trends,
+            "seconds": time.perf_counter() - t0}
+    print(json.dumps(line), flush=True)
+    for r in rows:
+        print(f"sigma {r['sigma']:<5} rho {r['rho']:<5} {r['router']:<9} rel_l2 {r['rel_l2']:.4e} "
+              f"max {r['max_abs']:.4e} density {r['density']:.4f} {r['ms']:.2f} ms", file=sys.stderr)
+    return 0
+
+
 # -------------------------------------------------------------------- ours
 
 def main():
     a = _args()
+    if a.stress:
+        return run_stress(a)
     from clustered_sparse_attention_flash_b200 import synth
     cfg = synth.CONFIGS[a.config]
     if a.heads is not None:

@@ -55,6 +55,7 @@ int check_params(const svgear_params* p) {
   if (!(p->rho >= 0.f && p->rho <= 1.f)) return SVGEAR_ERR_INVALID;
   if (std::isnan(p->scale) || std::isinf(p->scale)) return SVGEAR_ERR_INVALID;
   if (p->Ck > kMaxCkBits) return SVGEAR_ERR_UNSUPPORTED;
+  if (p->router < SVGEAR_ROUTE_ERROR || p->router > SVGEAR_ROUTE_ERROR_NOV) return SVGEAR_ERR_INVALID;
   return SVGEAR_OK;
 }
 
@@ -200,11 +201,14 @@ int svgear_block_error(const float* Qbar, const float* Kbar, const float* Vbar, 
                        void* stream) {
   int r = check_params(p);
   if (r) return r;
-  if (!Qbar || !Kbar || !Kp || !k_off || !key_scalars || !E || !M) return SVGEAR_ERR_INVALID;
+  if (!Qbar || !Kbar || !k_off || !E || !M) return SVGEAR_ERR_INVALID;
+  if (p->router != SVGEAR_ROUTE_MASS && !Kp) return SVGEAR_ERR_INVALID;
+  if (p->router == SVGEAR_ROUTE_ERROR && !key_scalars) return SVGEAR_ERR_INVALID;
   if (!aligned16(Qbar) || !aligned16(Kbar) || !aligned16(Kp)) return SVGEAR_ERR_INVALID;
   if (!ws || ws_bytes < block_error_ws_bytes(p->H, p->Cq, p->Ck, p->d, p->dtype)) return SVGEAR_ERR_WORKSPACE;
   return cuda_status(block_error_run(Qbar, Kbar, Vbar, Kp, Vp, k_off, key_scalars, p->dtype, p->H,
-                                     p->Nk, p->d, p->Cq, p->Ck, eff_scale(p), E, M, ws, S(stream)));
+                                     p->Nk, p->d, p->Cq, p->Ck, eff_scale(p), E, M, ws, S(stream),
+                                     p->router));
 }
 
 int svgear_route(const float* E, const int32_t* k_counts, const int32_t* q_counts,
@@ -295,7 +299,7 @@ int svgear_forward(const void* Q, const void* K, const void* V, const svgear_par
   mark(3);
   if (e == cudaSuccess)
     e = block_error_run(L.cent_q, L.cent_k, L.vbar, L.Kp, L.Vp, L.off_k, L.key_scalars, dt, H, Nk, d,
-                        Cq, Ck, sc, L.E, L.M, L.scratch, st);
+                        Cq, Ck, sc, L.E, L.M, L.scratch, st, p->router);
   mark(4);
   if (e == cudaSuccess)
     e = route_run(L.E, L.counts_k, L.counts_q, H, Nk, Cq, Ck, p->rho, L.mask, L.sel, L.n_sel,

@@ -13,6 +13,11 @@
 // This is exact algebra; the form keeps full relative accuracy when the
 // cluster is tight (u -> 0, v -> vbar) where a^2|vbar|^2 - 2ab vbar.v + b^2|v|^2
 // would cancel.  Logits never leave registers.
+//
+// Two ablation signals share the launch sequence: the value-agnostic error
+// (s1, s2, s3) = (0, 0, 1), i.e. eps^2 = (A - B)^2, and the estimated
+// attention mass of each key cluster, |k_c| A normalised over the row, which
+// needs only the centroid logits.
 #include <mutex>
 
 #include "../../include/svgear.h"
@@ -71,6 +76,31 @@ __global__ void __launch_bounds__(256) k_logit_max(const float* __restrict__ L, 
   if (lane == 0) M[row] = mx;
 }
 
+// Estimated attention mass: E[a][c] = |k_c| e^{L[a][c] - M[a]} / row sum over
+// the non-empty clusters (0 for empty ones).  One warp per (a, head); the row
+// sum is accumulated in float64.
+__global__ void __launch_bounds__(256) k_block_mass(const float* __restrict__ L, const float* __restrict__ M,
+                                                    const int32_t* __restrict__ k_off, int H, int Cq, int Ck,
+                                                    float* __restrict__ E) {
+  const int row = blockIdx.x * 8 + (threadIdx.x >> 5), lane = threadIdx.x & 31;
+  if (row >= H * Cq) return;
+  const int h = row / Cq;
+  const int32_t* off = k_off + (size_t)h * (Ck + 1);
+  const float* Lr = L + (size_t)row * Ck;
+  float* Er = E + (size_t)row * Ck;
+  const float m = M[row];
+  double sum = 0.0;
+  for (int c = lane; c < Ck; c += 32) {
+    const int n = off[c + 1] - off[c];
+    const float w = n > 0 ? (float)n * expf(Lr[c] - m) : 0.f;
+    Er[c] = w;
+    sum += (double)w;
+  }
+  for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+  const float inv = (float)(1.0 / sum);  // sum >= 1: the maximising cluster has n >= 1, e^0
+  for (int c = lane; c < Ck; c += 32) Er[c] *= inv;
+}
+
 // One block per (key cluster c, head); thread t owns query cluster a = t (+128k).
 // Keys of c stream through shared memory as k_j - kbar_c.
 template <typename T, int D>
@@ -80,7 +110,8 @@ __global__ void __launch_bounds__(128) k_block_error(const float* __restrict__ Q
                                                      const int32_t* __restrict__ k_off,
                                                      const float* __restrict__ ks, const float* __restrict__ L,
                                                      const float* __restrict__ M, int H, int Nk, int Cq,
-                                                     int Ck, float scale, float* __restrict__ E) {
+                                                     int Ck, float scale, int value_agnostic,
+                                                     float* __restrict__ E) {
   constexpr int KT = 32;
   __shared__ __align__(16) float dk[KT][D];
   __shared__ float sc[3][KT];
@@ -121,7 +152,7 @@ __global__ void __launch_bounds__(128) k_block_error(const float* __restrict__ Q
       }
       for (int e = threadIdx.x; e < 3 * nk; e += blockDim.x) {
         const int w = e / nk, r = e % nk;
-        sc[w][r] = ks[w * plane + (size_t)h * Nk + j0 + r];
+        sc[w][r] = value_agnostic ? (w == 2 ? 1.f : 0.f) : ks[w * plane + (size_t)h * Nk + j0 + r];
       }
       __syncthreads();
       if (act) {
@@ -156,24 +187,30 @@ cudaError_t block_error_run(const float* Qbar, const float* Kbar, const float* V
                             const void* Kp, const void* Vp, const int32_t* k_off,
                             const float* key_scalars, int dtype, int H, int Nk, int d, int Cq,
                             int Ck, float scale, float* E, float* M, void* ws, cudaStream_t st,
-                            bool allow_tc) {
+                            int router, bool allow_tc) {
   (void)Vbar; (void)Vp;  // their contribution enters through key_scalars
   float* L = static_cast<float*>(ws);
   const dim3 lg((Ck + 31) / 32, (Cq + 31) / 32, H);
   if (d == 128) { k_centroid_logits<128><<<lg, 256, 0, st>>>(Qbar, Kbar, Cq, Ck, scale, L); note_launch(); }
   else { k_centroid_logits<64><<<lg, 256, 0, st>>>(Qbar, Kbar, Cq, Ck, scale, L); note_launch(); }
   k_logit_max<<<(H * Cq + 7) / 8, 256, 0, st>>>(L, k_off, H, Cq, Ck, M); note_launch();
+  if (router == SVGEAR_ROUTE_MASS) {
+    k_block_mass<<<(H * Cq + 7) / 8, 256, 0, st>>>(L, M, k_off, H, Cq, Ck, E); note_launch();
+    return cudaGetLastError();
+  }
+  const int vagn = router == SVGEAR_ROUTE_ERROR_NOV;
   if (allow_tc && block_error_tc_supported(dtype, d, Cq, Nk)) {
     char* qhl = static_cast<char*>(ws) + align_up((size_t)H * Cq * Ck * sizeof(float), 256);
-    return block_error_tc_run(Qbar, Kp, k_off, key_scalars, L, M, H, Nk, d, Cq, Ck, scale, E, qhl, st);
+    return block_error_tc_run(Qbar, Kp, k_off, key_scalars, L, M, H, Nk, d, Cq, Ck, scale, E, qhl, st,
+                              vagn != 0);
   }
   dim3 g(Ck, H);
   if (dtype == DT_BF16) {
-    if (d == 128) { k_block_error<bf16, 128><<<g, 128, 0, st>>>(Qbar, Kbar, static_cast<const bf16*>(Kp), k_off, key_scalars, L, M, H, Nk, Cq, Ck, scale, E); note_launch(); }
-    else { k_block_error<bf16, 64><<<g, 128, 0, st>>>(Qbar, Kbar, static_cast<const bf16*>(Kp), k_off, key_scalars, L, M, H, Nk, Cq, Ck, scale, E); note_launch(); }
+    if (d == 128) { k_block_error<bf16, 128><<<g, 128, 0, st>>>(Qbar, Kbar, static_cast<const bf16*>(Kp), k_off, key_scalars, L, M, H, Nk, Cq, Ck, scale, vagn, E); note_launch(); }
+    else { k_block_error<bf16, 64><<<g, 128, 0, st>>>(Qbar, Kbar, static_cast<const bf16*>(Kp), k_off, key_scalars, L, M, H, Nk, Cq, Ck, scale, vagn, E); note_launch(); }
   } else {
-    if (d == 128) { k_block_error<float, 128><<<g, 128, 0, st>>>(Qbar, Kbar, static_cast<const float*>(Kp), k_off, key_scalars, L, M, H, Nk, Cq, Ck, scale, E); note_launch(); }
-    else { k_block_error<float, 64><<<g, 128, 0, st>>>(Qbar, Kbar, static_cast<const float*>(Kp), k_off, key_scalars, L, M, H, Nk, Cq, Ck, scale, E); note_launch(); }
+    if (d == 128) { k_block_error<float, 128><<<g, 128, 0, st>>>(Qbar, Kbar, static_cast<const float*>(Kp), k_off, key_scalars, L, M, H, Nk, Cq, Ck, scale, vagn, E); note_launch(); }
+    else { k_block_error<float, 64><<<g, 128, 0, st>>>(Qbar, Kbar, static_cast<const float*>(Kp), k_off, key_scalars, L, M, H, Nk, Cq, Ck, scale, vagn, E); note_launch(); }
   }
   return cudaGetLastError();
 }
@@ -213,7 +250,9 @@ extern "C" int svgear_block_error_noalloc(const float* Qbar, const float* Kbar, 
   using namespace svg;
   const int r = params_status(p);
   if (r != SVGEAR_OK) return r;
-  if (!Qbar || !Kbar || !Kp || !k_off || !key_scalars || !E || !M) return SVGEAR_ERR_INVALID;
+  if (!Qbar || !Kbar || !k_off || !E || !M) return SVGEAR_ERR_INVALID;
+  if (p->router != SVGEAR_ROUTE_MASS && !Kp) return SVGEAR_ERR_INVALID;
+  if (p->router == SVGEAR_ROUTE_ERROR && !key_scalars) return SVGEAR_ERR_INVALID;
   const uintptr_t mis = reinterpret_cast<uintptr_t>(Qbar) | reinterpret_cast<uintptr_t>(Kbar) |
                         reinterpret_cast<uintptr_t>(Kp);
   if (mis & 15u) return SVGEAR_ERR_INVALID;
@@ -224,6 +263,6 @@ extern "C" int svgear_block_error_noalloc(const float* Qbar, const float* Kbar, 
   const float scale = p->scale > 0.f ? p->scale : 1.0f / sqrtf((float)p->d);
   // the static scratch holds the centroid logits only: CUDA-core block error
   e = block_error_run(Qbar, Kbar, Vbar, Kp, Vp, k_off, key_scalars, p->dtype, p->H, p->Nk, p->d, p->Cq,
-                      p->Ck, scale, E, M, L, static_cast<cudaStream_t>(stream), false);
+                      p->Ck, scale, E, M, L, static_cast<cudaStream_t>(stream), p->router, false);
   return e == cudaSuccess ? SVGEAR_OK : SVGEAR_ERR_CUDA;
 }

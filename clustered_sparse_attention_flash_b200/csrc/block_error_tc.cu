@@ -15,6 +15,8 @@
 // order.  Block of 6 warps: warp 0 allocates tensor memory and issues MMAs,
 // warp 1 issues the TMA copies of the key tiles and stages the per-key
 // scalars, warps 2-5 are the epilogue (one TMEM lane = one query cluster).
+// For the value-agnostic ablation the staged scalars are (0, 0, 1), so each
+// key adds w^2 = (A - B_j)^2 / A^2.
 #include <cuda.h>
 
 #include <algorithm>
@@ -94,7 +96,7 @@ __global__ void __launch_bounds__(kBeThreads, 1)
     k_block_error_tc(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmk,
                      const int32_t* __restrict__ k_off, const float* __restrict__ ks,
                      const float* __restrict__ L, const float* __restrict__ M, int H, int Nk, int Cq, int Ck,
-                     float* __restrict__ E, int* status) {
+                     int value_agnostic, float* __restrict__ E, int* status) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const BeLay Ly = be_layout(D);
@@ -187,7 +189,7 @@ __global__ void __launch_bounds__(kBeThreads, 1)
                             part * kBeRows, h, q_full);
       }
       const size_t plane = (size_t)H * Nk;
-      const float* ks1 = ks + (size_t)h * Nk;
+      const float* ks1 = value_agnostic ? nullptr : ks + (size_t)h * Nk;
       for (int t = 0; t < ntiles; ++t) {
         const int s = t % kBeStages;
         const bool ok = tc::mbar_wait_warp(empty + s, ((t / kBeStages) & 1) ^ 1, abort_flag, status);
@@ -203,7 +205,8 @@ __global__ void __launch_bounds__(kBeThreads, 1)
         for (int i = lane; i < kBeKeys; i += 32) {
           const int j = j0 + i;
           float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-          if (j < ke) v = make_float4(ks1[j], ks1[plane + j], ks1[2 * plane + j], 0.f);
+          if (j < ke)
+            v = ks1 ? make_float4(ks1[j], ks1[plane + j], ks1[2 * plane + j], 0.f) : make_float4(0.f, 0.f, 1.f, 0.f);
           sc[i] = v;
         }
         __syncwarp();
@@ -325,7 +328,7 @@ static int pick_blocks_per_head(int H, int Nk) {
 template <int D>
 static cudaError_t be_launch(const float* Qbar, const bf16* Kp, const int32_t* k_off, const float* ks,
                              const float* L, const float* M, int H, int Nk, int Cq, int Ck, float scale,
-                             float* E, bf16* qhl, cudaStream_t st) {
+                             float* E, bf16* qhl, cudaStream_t st, int vagn) {
   k_prep_qhl<D><<<H, 256, 0, st>>>(Qbar, Cq, scale, qhl);
   note_launch();
   CUtensorMap tmq, tmk;
@@ -335,21 +338,21 @@ static cudaError_t be_launch(const float* Qbar, const bf16* Kp, const int32_t* k
   cudaError_t e = cudaFuncSetAttribute(k_block_error_tc<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
   const int G = pick_blocks_per_head(H, Nk);
-  k_block_error_tc<D><<<dim3(G, H), kBeThreads, smem, st>>>(tmq, tmk, k_off, ks, L, M, H, Nk, Cq, Ck, E,
-                                                             status_word());
+  k_block_error_tc<D><<<dim3(G, H), kBeThreads, smem, st>>>(tmq, tmk, k_off, ks, L, M, H, Nk, Cq, Ck, vagn,
+                                                             E, status_word());
   note_launch();
   return cudaGetLastError();
 }
 
 cudaError_t block_error_tc_run(const float* Qbar, const void* Kp, const int32_t* k_off, const float* ks,
                                const float* L, const float* M, int H, int Nk, int d, int Cq, int Ck,
-                               float scale, float* E, void* ws, cudaStream_t st) {
+                               float scale, float* E, void* ws, cudaStream_t st, bool value_agnostic) {
   if ((reinterpret_cast<uintptr_t>(Kp) & 15u) || (reinterpret_cast<uintptr_t>(ws) & 15u))
     return cudaErrorInvalidValue;
   const bf16* kp = static_cast<const bf16*>(Kp);
   bf16* qhl = static_cast<bf16*>(ws);
-  if (d == 128) return be_launch<128>(Qbar, kp, k_off, ks, L, M, H, Nk, Cq, Ck, scale, E, qhl, st);
-  return be_launch<64>(Qbar, kp, k_off, ks, L, M, H, Nk, Cq, Ck, scale, E, qhl, st);
+  if (d == 128) return be_launch<128>(Qbar, kp, k_off, ks, L, M, H, Nk, Cq, Ck, scale, E, qhl, st, value_agnostic ? 1 : 0);
+  return be_launch<64>(Qbar, kp, k_off, ks, L, M, H, Nk, Cq, Ck, scale, E, qhl, st, value_agnostic ? 1 : 0);
 }
 
 }  // namespace svg

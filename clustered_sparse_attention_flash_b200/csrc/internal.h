@@ -46,14 +46,14 @@ cudaError_t block_error_run(const float* Qbar, const float* Kbar, const float* V
                             const void* Kp, const void* Vp, const int32_t* k_off,
                             const float* key_scalars, int dtype, int H, int Nk, int d, int Cq,
                             int Ck, float scale, float* E, float* M, void* ws, cudaStream_t st,
-                            bool allow_tc = true);
+                            int router = 0, bool allow_tc = true);
 // tensor-core kernel (block_error_tc.cu); L and M already computed
 bool block_error_tc_shape_ok(int dtype, int d, int Cq);
 bool block_error_tc_supported(int dtype, int d, int Cq, int Nk);
 size_t block_error_tc_ws_bytes(int H, int d);
 cudaError_t block_error_tc_run(const float* Qbar, const void* Kp, const int32_t* k_off, const float* ks,
                                const float* L, const float* M, int H, int Nk, int d, int Cq, int Ck,
-                               float scale, float* E, void* ws, cudaStream_t st);
+                               float scale, float* E, void* ws, cudaStream_t st, bool value_agnostic);
 
 // ---- routing
 cudaError_t route_run(const float* E, const int32_t* k_counts, const int32_t* q_counts,

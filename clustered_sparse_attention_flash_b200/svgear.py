@@ -25,6 +25,9 @@ SVGEAR_ERR_TIMEOUT = -4
 SVGEAR_ERR_WORKSPACE = -5
 SVGEAR_F32 = 0
 SVGEAR_BF16 = 1
+SVGEAR_ROUTE_ERROR = 0
+SVGEAR_ROUTE_MASS = 1
+SVGEAR_ROUTE_ERROR_NOV = 2
 
 
 class SvgearError(RuntimeError):
@@ -37,7 +40,7 @@ class svgear_params(ctypes.Structure):
     _fields_ = [("H", ctypes.c_int), ("Nq", ctypes.c_int), ("Nk", ctypes.c_int),
                 ("d", ctypes.c_int), ("Cq", ctypes.c_int), ("Ck", ctypes.c_int),
                 ("iters", ctypes.c_int), ("rho", ctypes.c_float), ("scale", ctypes.c_float),
-                ("dtype", ctypes.c_int)]
+                ("dtype", ctypes.c_int), ("router", ctypes.c_int)]
 
 
 class svgear_stats(ctypes.Structure):
@@ -138,8 +141,9 @@ def _check(fn: str, code: int) -> None:
         raise SvgearError(fn, code)
 
 
-def params(H, Nq, Nk, d, Cq, Ck, iters, rho, scale=0.0, dtype=SVGEAR_BF16) -> svgear_params:
-    return svgear_params(H, Nq, Nk, d, Cq, Ck, iters, rho, scale, dtype)
+def params(H, Nq, Nk, d, Cq, Ck, iters, rho, scale=0.0, dtype=SVGEAR_BF16,
+           router=SVGEAR_ROUTE_ERROR) -> svgear_params:
+    return svgear_params(H, Nq, Nk, d, Cq, Ck, iters, rho, scale, dtype, router)
 
 
 # ----------------------------------------------------------------- entries
@@ -285,13 +289,14 @@ def view_tensors(p: svgear_params, ws) -> Dict[str, "object"]:
 
 
 def forward(Q, K, V, Cq: int, Ck: int, iters: int, rho: float, scale: float = 0.0,
-            init_q=None, init_k=None, ws=None, stream=None, stats: bool = False):
+            init_q=None, init_k=None, ws=None, stream=None, stats: bool = False,
+            router: int = SVGEAR_ROUTE_ERROR):
     """Allocate O (and the workspace unless given) and run svgear_forward.
     Returns (O, ws, params, stats-dict or None)."""
     import torch
     H, Nq, d = Q.shape
     Nk = K.shape[1]
-    p = params(H, Nq, Nk, d, Cq, Ck, iters, rho, scale, dtype_code(Q))
+    p = params(H, Nq, Nk, d, Cq, Ck, iters, rho, scale, dtype_code(Q), router)
     need = svgear_workspace_size(p)
     if need == 0:
         raise SvgearError("svgear_workspace_size", SVGEAR_ERR_INVALID)

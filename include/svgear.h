@@ -61,6 +61,25 @@ typedef enum {
 
 typedef enum { SVGEAR_F32 = 0, SVGEAR_BF16 = 1 } svgear_dtype;
 
+/* What svgear_block_error stores in E, i.e. the signal the router ranks key
+ * clusters by.  Only SVGEAR_ROUTE_ERROR is the method; the other two are
+ * ablations that swap the ranking signal and keep every other step.
+ *   SVGEAR_ROUTE_ERROR      value-aware error-to-cost ratio (review step (2),
+ *                           gist.science 2.B): the default, 0.
+ *   SVGEAR_ROUTE_MASS       estimated attention mass of each key cluster for
+ *                           the query centroid, |k_c| e^{s qbar_a.kbar_c},
+ *                           normalised to sum 1 over the non-empty clusters of
+ *                           the row -- a score-based router in the manner of
+ *                           the top-p selectors the pages compare against.
+ *   SVGEAR_ROUTE_ERROR_NOV  value-agnostic error: eps^2 without the values,
+ *                           (e^{s qbar_a.kbar_c} - e^{s qbar_a.k_j})^2, same
+ *                           shift and per-key average as the default. */
+typedef enum {
+  SVGEAR_ROUTE_ERROR = 0,
+  SVGEAR_ROUTE_MASS = 1,
+  SVGEAR_ROUTE_ERROR_NOV = 2
+} svgear_router;
+
 /* Operator hyper-parameters of one attention layer. */
 typedef struct {
   int H;        /* heads (independent problems) */
@@ -72,6 +91,8 @@ typedef struct {
                    most floor(rho * Nk) keys exactly */
   float scale;  /* softmax scale; <= 0 selects 1/sqrt(d) */
   int dtype;    /* svgear_dtype of Q, K, V and the output */
+  int router;   /* svgear_router: what E ranks by; 0 (zero-initialised
+                   params) is the method's value-aware error */
 } svgear_params;
 
 /* Per-stage device times of one svgear_forward call (CUDA events). */
@@ -161,6 +182,14 @@ SVGEAR_API int svgear_permute(const void* X, int dtype, const int32_t* labels, i
  * E is the pages' error-to-cost ratio times the positive per-row factor
  * exp(-2 M_a), which keeps it in float32 range and leaves the routing order
  * unchanged.  Empty key clusters get E = 0.
+ * p->router selects an ablation instead (M as above in every mode):
+ *   SVGEAR_ROUTE_MASS:      E[h][a][c] = |k_c| e^{s qbar_a.kbar_c - M_a} /
+ *                           sum over non-empty c' of the same; Kp, Vp and
+ *                           key_scalars are not read.
+ *   SVGEAR_ROUTE_ERROR_NOV: eps^2(a,j) = (e^{s qbar_a.kbar_c} -
+ *                           e^{s qbar_a.k_j})^2 in the formula above; Vbar,
+ *                           Vp and key_scalars are not read.
+ * Router values outside svgear_router return SVGEAR_ERR_INVALID.
  *   Qbar [H,Cq,d], Kbar/Vbar [H,Ck,d] float32; Kp/Vp [H,Nk,d] dtype (keys in
  *   cluster order); k_off [H,Ck+1]; key_scalars [3,H,Nk] from svgear_permute.
  * ------------------------------------------------------------------------- */

@@ -1,6 +1,7 @@
 """The C-ABI library loads and exports every entry point its header declares;
 host-side validation answers without touching a GPU."""
 import ctypes
+import os
 
 import pytest
 
@@ -20,6 +21,25 @@ def test_every_header_symbol_is_exported(L):
     for n in names:
         assert hasattr(L, n), n
     assert set(names) == set(sv._SIGS), set(names) ^ set(sv._SIGS)
+
+
+def test_params_struct_matches_header(tmp_path):
+    """The ctypes mirror of svgear_params has the C struct's size and field
+    offsets (compiled with the host C compiler against the header)."""
+    import shutil
+    import subprocess
+    cc = shutil.which("gcc") or shutil.which("cc")
+    if cc is None:
+        pytest.skip("no host C compiler")
+    fields = [n for n, _ in sv.svgear_params._fields_]
+    src = tmp_path / "p.c"
+    src.write_text('#include <stdio.h>\n#include <stddef.h>\n#include "svgear.h"\nint main(void){printf("%zu", sizeof(svgear_params));'
+                   + "".join(f'printf(" %zu", offsetof(svgear_params, {n}));' for n in fields) + "return 0;}\n")
+    exe = tmp_path / "p"
+    subprocess.run([cc, "-I", os.path.dirname(sv.HEADER), str(src), "-o", str(exe)], check=True)
+    got = [int(x) for x in subprocess.run([str(exe)], capture_output=True, text=True, check=True).stdout.split()]
+    assert got[0] == ctypes.sizeof(sv.svgear_params)
+    assert got[1:] == [getattr(sv.svgear_params, n).offset for n in fields]
 
 
 def test_version_and_status_strings(L):
@@ -56,3 +76,10 @@ def test_validation_rejects_before_any_launch(L):
     assert f(18, 16, 16, ctypes.byref(p), None, None, 16, 16, 1 << 30, None, None) == sv.SVGEAR_ERR_INVALID
     assert L.svgear_kmeans(16, 0, 1, 10, 64, 0, 1, None, 16, 16, 16, 16, 1 << 20, None) == sv.SVGEAR_ERR_INVALID
     assert L.svgear_route(None, None, None, ctypes.byref(p), None, None, None, None, None) == sv.SVGEAR_ERR_INVALID
+    # routing signal outside svgear_router
+    for r in (-1, 3):
+        bad = sv.params(1, 256, 256, 64, 4, 8, 2, 0.5, router=r)
+        assert f(16, 16, 16, ctypes.byref(bad), None, None, 16, 16, 1 << 30, None, None) == sv.SVGEAR_ERR_INVALID
+        assert sv.svgear_workspace_size(bad) == 0
+    for r in (sv.SVGEAR_ROUTE_MASS, sv.SVGEAR_ROUTE_ERROR_NOV):
+        assert sv.svgear_workspace_size(sv.params(1, 256, 256, 64, 4, 8, 2, 0.5, router=r)) > 0
