@@ -339,6 +339,43 @@ def route(E, k_counts, q_counts, rho):
     return mask, sel, pairs
 
 
+def route_global_budget(rho, Nq: int, Nk: int) -> int:
+    """floor(rho * N_q * N_k) pairs, rho as the float32 the operator receives,
+    in exact rational arithmetic."""
+    from fractions import Fraction
+    return int(math.floor(Fraction(float(np.float32(rho))) * Nq * Nk))
+
+
+def route_global(E, M, k_counts, q_counts, rho):
+    """Global-budget routing (the knapsack form of [DE] 2.B taken over all
+    blocks of a head at once): every block (a, c) with |q_a| > 0 and
+    |k_c| > 0 is an item of cost |q_a| |k_c| and value the unshifted
+    error-to-cost ratio E[a, c] exp(2 M_a); items in ratio order (descending;
+    equal ratios: smaller a * Ck + c first); the longest prefix whose total
+    cost fits floor(rho N_q N_k) is routed.  Ratios are compared as
+    log E + 2 M (E = 0 is -inf).  Returns (mask, sel per row in that row's
+    order, exec_pairs) like route."""
+    E = _f64(E)
+    M = _f64(M)
+    k_counts = np.asarray(k_counts, dtype=np.int64)
+    q_counts = np.asarray(q_counts, dtype=np.int64)
+    Cq, Ck = E.shape
+    budget = route_global_budget(rho, int(q_counts.sum()), int(k_counts.sum()))
+    with np.errstate(divide="ignore"):
+        key = np.log(np.maximum(E, 0.0)) + 2.0 * M[:, None]
+    valid = (q_counts[:, None] > 0) & (k_counts[None, :] > 0)
+    idx = np.arange(Cq * Ck)
+    order = np.lexsort((idx, -key.ravel()))
+    order = order[valid.ravel()[order]]
+    cost = (q_counts[:, None] * k_counts[None, :]).ravel()[order]
+    n = int(np.searchsorted(np.cumsum(cost), budget, side="right"))
+    mask = np.zeros((Cq, Ck), dtype=np.uint8)
+    mask.ravel()[order[:n]] = 1
+    sel = [order[:n][order[:n] // Ck == a] % Ck for a in range(Cq)]
+    pairs = int(cost[:n].sum())
+    return mask, sel, pairs
+
+
 # --------------------------------------------------------------------------
 # (4) hybrid attention: exact routed blocks + centroid compensation, one
 #     softmax                                [R] step (4); [DE] 2.A; [IT] 2.A
@@ -392,16 +429,24 @@ def dense_attention(Q, K, V, scale: float) -> np.ndarray:
 # --------------------------------------------------------------------------
 
 def forward(Q, K, V, Cq: int, Ck: int, iters: int, rho, scale: float,
-            init_q, init_k, router: str = "error") -> Dict[str, object]:
+            init_q, init_k, router: str = "error",
+            budget: str = "row") -> Dict[str, object]:
     """All steps of one head in order; returns every intermediate.  `router`
-    names the routing signal (ROUTERS; "error" is the method)."""
+    names the routing signal (ROUTERS; "error" is the method); `budget` is
+    "row" (floor(rho N_k) keys per query cluster, the method) or "global"
+    (route_global)."""
     Qbar, lq, cq = kmeans(Q, Cq, iters, init_q)
     Kbar, lk, ck = kmeans(K, Ck, iters, init_k)
     perm_q, off_q, _ = permute(lq, Cq)
     perm_k, off_k, _ = permute(lk, Ck)
     Vbar = value_centroids(V, lk, Ck)
     E, M = routing_signal(router, Qbar, Kbar, Vbar, K, V, lk, ck, scale)
-    mask, sel, pairs = route(E, ck, cq, rho)
+    if budget == "row":
+        mask, sel, pairs = route(E, ck, cq, rho)
+    elif budget == "global":
+        mask, sel, pairs = route_global(E, M, ck, cq, rho)
+    else:
+        raise ValueError(budget)
     O = hybrid_attention(Q, K, V, lq, lk, Kbar, Vbar, ck, mask, scale)
     return dict(Qbar=Qbar, Kbar=Kbar, Vbar=Vbar, q_labels=lq, k_labels=lk,
                 q_counts=cq, k_counts=ck, perm_q=perm_q, perm_k=perm_k,

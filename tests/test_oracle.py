@@ -386,12 +386,78 @@ def test_hybrid_rho_zero_is_biased_centroid_attention():
     np.testing.assert_allclose(out["O"], want, rtol=1e-10, atol=1e-12)
 
 
+# ------------------------------------------------------- global budget ----
+
+def test_route_global_worked_example():
+    """Two query clusters (sizes 2, 1), three key clusters (sizes 1, 2, 3):
+    18 pairs, rho = 10/18 gives a budget of 10.  With M = (0, ln 2) the
+    unshifted ratios are row 0: .5 .2 .1 and row 1 (x4): .04 .6 .16, so the
+    order is (1,1) .6 cost 2, (0,0) .5 cost 2, (0,1) .2 cost 4, (1,2) .16
+    cost 3, (0,2) .1 cost 6, (1,0) .04 cost 1; running costs 2 4 8 11 ...
+    The first three fit; (1,0) would fit the 2 left over but lies after the
+    first item that does not, so the prefix stops there."""
+    E = np.array([[0.5, 0.2, 0.1], [0.01, 0.15, 0.04]])
+    M = np.array([0.0, math.log(2.0)])
+    kc, qc = np.array([1, 2, 3]), np.array([2, 1])
+    rho = np.float32(10 / 18)
+    assert ora.route_global_budget(rho, 3, 6) == 10
+    mask, sel, pairs = ora.route_global(E, M, kc, qc, rho)
+    np.testing.assert_array_equal(mask, [[1, 1, 0], [0, 1, 0]])
+    assert [list(x) for x in sel] == [[0, 1], [1]]
+    assert pairs == 8
+    # the shift enters with the sign that undoes exp(-2 M): flipping it
+    # reorders row 1 below row 0 and must change the routing
+    m2, _, _ = ora.route_global(E, -M, kc, qc, rho)
+    assert not np.array_equal(m2, mask)
+
+
+def test_route_global_budget_is_exact():
+    """float32(0.1) = 0.100000001490116119384765625; times 75,600^2 =
+    5,715,360,000 gives 571,536,008.5166..., floor 571,536,008."""
+    assert ora.route_global_budget(0.1, 75600, 75600) == 571536008
+    assert ora.route_global_budget(1.0, 75600, 75600) == 75600 * 75600
+    assert ora.route_global_budget(0.0, 10, 10) == 0
+
+
+def test_route_global_depends_on_unshifted_ratio_only():
+    """Moving exp(2 M_a) into E (and M to 0) leaves the routing unchanged."""
+    rng = np.random.default_rng(31)
+    Cq, Ck = 7, 11
+    E = rng.random((Cq, Ck)) * np.exp(rng.normal(size=(Cq, Ck)))
+    M = rng.normal(size=Cq)
+    kc = rng.integers(0, 9, Ck); kc[0] = 3
+    qc = rng.integers(0, 9, Cq); qc[0] = 2
+    for rho in (0.05, 0.3, 0.7):
+        a = ora.route_global(E, M, kc, qc, rho)
+        b = ora.route_global(E * np.exp(2 * M)[:, None], np.zeros(Cq), kc, qc, rho)
+        np.testing.assert_array_equal(a[0], b[0])
+        assert a[2] == b[2] <= ora.route_global_budget(rho, qc.sum(), kc.sum())
+
+
+def test_route_global_extremes():
+    rng = np.random.default_rng(32)
+    E = rng.random((4, 6)); M = rng.normal(size=4)
+    kc = np.array([3, 0, 2, 5, 1, 4]); qc = np.array([2, 0, 7, 1])
+    mask, _, pairs = ora.route_global(E, M, kc, qc, 1.0)
+    np.testing.assert_array_equal(mask, (qc[:, None] > 0) & (kc[None, :] > 0))
+    assert pairs == qc.sum() * kc.sum()
+    mask, sel, pairs = ora.route_global(E, M, kc, qc, 0.0)
+    assert mask.sum() == 0 and pairs == 0 and all(len(x) == 0 for x in sel)
+
+
 @pytest.mark.parametrize("router", ["mass", "error_nov"])
 def test_ablation_routers_rho_one_is_dense(router):
     """Whatever the ranking signal, rho = 1 routes every non-empty cluster."""
     Q, K, V, Cq, Ck = _small_case(15)
     s = 1 / math.sqrt(8)
     out = ora.forward(Q, K, V, Cq, Ck, 3, 1.0, s, Q[:Cq], K[:Ck], router=router)
+    np.testing.assert_allclose(out["O"], _sdpa64(Q, K, V, s), rtol=1e-10, atol=1e-12)
+
+
+def test_global_budget_forward_rho_one_is_dense():
+    Q, K, V, Cq, Ck = _small_case(16)
+    s = 1 / math.sqrt(8)
+    out = ora.forward(Q, K, V, Cq, Ck, 3, 1.0, s, Q[:Cq], K[:Ck], budget="global")
     np.testing.assert_allclose(out["O"], _sdpa64(Q, K, V, s), rtol=1e-10, atol=1e-12)
 
 
