@@ -293,7 +293,8 @@ def run_stress(a):
     """Relative L2 and max error of the operator's output against dense
     attention on the stress workload (H=16, N=32,768, d=128, Cq=64, Ck=512),
     for each within-center noise sigma and density budget rho, with the
-    method's error-aware router and the two ablation signals.  The yardstick is
+    method's error-aware router, the two ablation signals, and the
+    error-aware signal under one global budget per head.  The yardstick is
     float32 dense attention on the GPU; rows of it are checked in float64."""
     from clustered_sparse_attention_flash_b200 import synth
     base = synth.CONFIGS["stress"]
@@ -309,8 +310,9 @@ def run_stress(a):
     torch.backends.cudnn.allow_tf32 = False
     dev = torch.device("cuda", 0)
     s = 1.0 / math.sqrt(base.d)
-    routers = (("error", sv.SVGEAR_ROUTE_ERROR), ("mass", sv.SVGEAR_ROUTE_MASS),
-               ("error_nov", sv.SVGEAR_ROUTE_ERROR_NOV))
+    G = sv.SVGEAR_BUDGET_GLOBAL
+    routers = (("error", sv.SVGEAR_ROUTE_ERROR, 0), ("mass", sv.SVGEAR_ROUTE_MASS, 0),
+               ("error_nov", sv.SVGEAR_ROUTE_ERROR_NOV, 0), ("error_global", sv.SVGEAR_ROUTE_ERROR, G))
     rows = []
     yard = {}
     t0 = time.perf_counter()
@@ -325,10 +327,10 @@ def run_stress(a):
         yard[sg] = float((ref[0, :256].double() - r64).abs().max())
         nref = float(torch.linalg.vector_norm(ref.double()))
         ws = None
-        for rname, rcode in routers:
+        for rname, rcode, bcode in routers:
             for rho in rhos:
                 O, ws, p, st = sv.forward(dQ, dK, dV, base.Cq, base.Ck, base.iters, rho, s, diq, dik,
-                                          ws=ws, stats=True, router=rcode)
+                                          ws=ws, stats=True, router=rcode, budget=bcode)
                 if sv.svgear_get_status() != sv.SVGEAR_OK:
                     raise RuntimeError("device status not OK")
                 d = O.float() - ref
@@ -350,7 +352,9 @@ def run_stress(a):
         # ... and must not rise as the budget grows (fixed sigma)
         "nonincreasing_in_rho": {str(sg): _nonincreasing([err(sg, rho) for rho in rhos]) for sg in sigmas},
         "error_router_best": {f"{sg}/{rho}": min(("error", "mass", "error_nov"), key=lambda r: err(sg, rho, r))
-                              for sg in sigmas for rho in rhos},
+                              for sg in sigmas for rho in rhos if rho < 1.0},
+        "global_budget_better": {f"{sg}/{rho}": err(sg, rho, "error_global") < err(sg, rho)
+                                 for sg in sigmas for rho in rhos if rho < 1.0},
     }
     line = {"stress": True, "workload": _workload(base, "swept"), "sigmas": sigmas, "rhos": rhos,
             "yardstick": "float32 dense attention on the GPU (TF32 off) from the same bf16 inputs",
@@ -358,7 +362,7 @@ def run_stress(a):
             "seconds": time.perf_counter() - t0}
     print(json.dumps(line), flush=True)
     for r in rows:
-        print(f"sigma {r['sigma']:<5} rho {r['rho']:<5} {r['router']:<9} rel_l2 {r['rel_l2']:.4e} "
+        print(f"sigma {r['sigma']:<5} rho {r['rho']:<5} {r['router']:<12} rel_l2 {r['rel_l2']:.4e} "
               f"max {r['max_abs']:.4e} density {r['density']:.4f} {r['ms']:.2f} ms", file=sys.stderr)
     return 0
 

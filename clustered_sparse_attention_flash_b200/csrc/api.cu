@@ -56,6 +56,9 @@ int check_params(const svgear_params* p) {
   if (std::isnan(p->scale) || std::isinf(p->scale)) return SVGEAR_ERR_INVALID;
   if (p->Ck > kMaxCkBits) return SVGEAR_ERR_UNSUPPORTED;
   if (p->router < SVGEAR_ROUTE_ERROR || p->router > SVGEAR_ROUTE_ERROR_NOV) return SVGEAR_ERR_INVALID;
+  if (p->budget != SVGEAR_BUDGET_ROW && p->budget != SVGEAR_BUDGET_GLOBAL) return SVGEAR_ERR_INVALID;
+  if (p->budget == SVGEAR_BUDGET_GLOBAL && (unsigned long long)p->Nq * (unsigned long long)p->Nk >= (1ull << 62))
+    return SVGEAR_ERR_UNSUPPORTED;
   return SVGEAR_OK;
 }
 
@@ -221,6 +224,17 @@ int svgear_route(const float* E, const int32_t* k_counts, const int32_t* q_count
                                n_sel, exec_pairs, S(stream)));
 }
 
+int svgear_route_global(const float* E, const float* M, const int32_t* k_counts, const int32_t* q_counts,
+                        const svgear_params* p, uint8_t* mask, int32_t* sel, int32_t* n_sel,
+                        int64_t* exec_pairs, void* stream) {
+  int r = check_params(p);
+  if (r) return r;
+  if (!E || !M || !k_counts || !q_counts || !mask || !sel || !n_sel || !exec_pairs) return SVGEAR_ERR_INVALID;
+  if ((unsigned long long)p->Nq * (unsigned long long)p->Nk >= (1ull << 62)) return SVGEAR_ERR_UNSUPPORTED;
+  return cuda_status(route_run(E, k_counts, q_counts, p->H, p->Nk, p->Cq, p->Ck, p->rho, mask, sel,
+                               n_sel, exec_pairs, S(stream), M, p->Nq));
+}
+
 size_t svgear_hybrid_attn_workspace_size(const svgear_params* p) {
   if (check_params(p)) return 0;
   return attn_ws_bytes(p->H, p->Nq, p->Nk, p->d, p->Cq, p->Ck);
@@ -303,7 +317,7 @@ int svgear_forward(const void* Q, const void* K, const void* V, const svgear_par
   mark(4);
   if (e == cudaSuccess)
     e = route_run(L.E, L.counts_k, L.counts_q, H, Nk, Cq, Ck, p->rho, L.mask, L.sel, L.n_sel,
-                  L.exec_pairs, st);
+                  L.exec_pairs, st, p->budget == SVGEAR_BUDGET_GLOBAL ? L.M : nullptr, Nq);
   mark(5);
   if (e == cudaSuccess)
     e = attn_run(L.Qp, L.Kp, L.Vp, L.off_q, L.off_k, L.perm_q, L.cent_k, L.vbar, L.sel, L.n_sel, dt,

@@ -58,7 +58,10 @@ cudaError_t block_error_tc_run(const float* Qbar, const void* Kp, const int32_t*
 // ---- routing
 cudaError_t route_run(const float* E, const int32_t* k_counts, const int32_t* q_counts,
                       int H, int Nk, int Cq, int Ck, float rho, uint8_t* mask, int32_t* sel,
-                      int32_t* n_sel, int64_t* exec_pairs, cudaStream_t st);
+                      int32_t* n_sel, int64_t* exec_pairs, cudaStream_t st,
+                      const float* M_global = nullptr, int Nq = 0);
+// floor(rho * Nq * Nk) in exact integer arithmetic (global budget, pairs)
+long long route_global_budget(float rho, long long Nq, long long Nk);
 
 // ---- hybrid attention
 size_t attn_ws_bytes(int H, int Nq, int Nk, int d, int Cq, int Ck);

@@ -28,6 +28,8 @@ SVGEAR_BF16 = 1
 SVGEAR_ROUTE_ERROR = 0
 SVGEAR_ROUTE_MASS = 1
 SVGEAR_ROUTE_ERROR_NOV = 2
+SVGEAR_BUDGET_ROW = 0
+SVGEAR_BUDGET_GLOBAL = 1
 
 
 class SvgearError(RuntimeError):
@@ -40,7 +42,7 @@ class svgear_params(ctypes.Structure):
     _fields_ = [("H", ctypes.c_int), ("Nq", ctypes.c_int), ("Nk", ctypes.c_int),
                 ("d", ctypes.c_int), ("Cq", ctypes.c_int), ("Ck", ctypes.c_int),
                 ("iters", ctypes.c_int), ("rho", ctypes.c_float), ("scale", ctypes.c_float),
-                ("dtype", ctypes.c_int), ("router", ctypes.c_int)]
+                ("dtype", ctypes.c_int), ("router", ctypes.c_int), ("budget", ctypes.c_int)]
 
 
 class svgear_stats(ctypes.Structure):
@@ -81,6 +83,7 @@ _SIGS = {
     "svgear_block_error": (_I, [_P, _P, _P, _P, _P, _P, _P, _PP, _P, _P, _P, _SZ, _P]),
     "svgear_block_error_noalloc": (_I, [_P, _P, _P, _P, _P, _P, _P, _PP, _P, _P, _P]),
     "svgear_route": (_I, [_P, _P, _P, _PP, _P, _P, _P, _P, _P]),
+    "svgear_route_global": (_I, [_P, _P, _P, _P, _PP, _P, _P, _P, _P, _P]),
     "svgear_hybrid_attn_workspace_size": (_SZ, [_PP]),
     "svgear_hybrid_attn": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _PP, _P, _P, _SZ, _P]),
     "svgear_workspace_size": (_SZ, [_PP]),
@@ -142,8 +145,8 @@ def _check(fn: str, code: int) -> None:
 
 
 def params(H, Nq, Nk, d, Cq, Ck, iters, rho, scale=0.0, dtype=SVGEAR_BF16,
-           router=SVGEAR_ROUTE_ERROR) -> svgear_params:
-    return svgear_params(H, Nq, Nk, d, Cq, Ck, iters, rho, scale, dtype, router)
+           router=SVGEAR_ROUTE_ERROR, budget=SVGEAR_BUDGET_ROW) -> svgear_params:
+    return svgear_params(H, Nq, Nk, d, Cq, Ck, iters, rho, scale, dtype, router, budget)
 
 
 # ----------------------------------------------------------------- entries
@@ -208,6 +211,12 @@ def svgear_block_error_noalloc(Qbar, Kbar, Vbar, Kp, Vp, k_off, key_scalars, p, 
 def svgear_route(E, k_counts, q_counts, p, mask, sel, n_sel, exec_pairs, stream=None):
     _check("svgear_route", lib().svgear_route(
         _ptr(E), _ptr(k_counts), _ptr(q_counts), ctypes.byref(p), _ptr(mask), _ptr(sel),
+        _ptr(n_sel), _ptr(exec_pairs), _stream(stream)))
+
+
+def svgear_route_global(E, M, k_counts, q_counts, p, mask, sel, n_sel, exec_pairs, stream=None):
+    _check("svgear_route_global", lib().svgear_route_global(
+        _ptr(E), _ptr(M), _ptr(k_counts), _ptr(q_counts), ctypes.byref(p), _ptr(mask), _ptr(sel),
         _ptr(n_sel), _ptr(exec_pairs), _stream(stream)))
 
 
@@ -290,13 +299,13 @@ def view_tensors(p: svgear_params, ws) -> Dict[str, "object"]:
 
 def forward(Q, K, V, Cq: int, Ck: int, iters: int, rho: float, scale: float = 0.0,
             init_q=None, init_k=None, ws=None, stream=None, stats: bool = False,
-            router: int = SVGEAR_ROUTE_ERROR):
+            router: int = SVGEAR_ROUTE_ERROR, budget: int = SVGEAR_BUDGET_ROW):
     """Allocate O (and the workspace unless given) and run svgear_forward.
     Returns (O, ws, params, stats-dict or None)."""
     import torch
     H, Nq, d = Q.shape
     Nk = K.shape[1]
-    p = params(H, Nq, Nk, d, Cq, Ck, iters, rho, scale, dtype_code(Q), router)
+    p = params(H, Nq, Nk, d, Cq, Ck, iters, rho, scale, dtype_code(Q), router, budget)
     need = svgear_workspace_size(p)
     if need == 0:
         raise SvgearError("svgear_workspace_size", SVGEAR_ERR_INVALID)

@@ -80,6 +80,13 @@ typedef enum {
   SVGEAR_ROUTE_ERROR_NOV = 2
 } svgear_router;
 
+/* How svgear_forward spends the density budget.
+ *   SVGEAR_BUDGET_ROW     floor(rho * Nk) keys for every query cluster
+ *                         (review step (3)): the default, 0.
+ *   SVGEAR_BUDGET_GLOBAL  one budget of floor(rho * Nq * Nk) query-key pairs
+ *                         per head over all blocks (svgear_route_global). */
+typedef enum { SVGEAR_BUDGET_ROW = 0, SVGEAR_BUDGET_GLOBAL = 1 } svgear_budget;
+
 /* Operator hyper-parameters of one attention layer. */
 typedef struct {
   int H;        /* heads (independent problems) */
@@ -93,6 +100,8 @@ typedef struct {
   int dtype;    /* svgear_dtype of Q, K, V and the output */
   int router;   /* svgear_router: what E ranks by; 0 (zero-initialised
                    params) is the method's value-aware error */
+  int budget;   /* svgear_budget: per query cluster (0) or per head (1);
+                   read by svgear_forward only */
 } svgear_params;
 
 /* Per-stage device times of one svgear_forward call (CUDA events). */
@@ -241,6 +250,23 @@ SVGEAR_API int svgear_route(const float* E, const int32_t* k_counts, const int32
                  int64_t* exec_pairs, void* stream);
 
 /* ---------------------------------------------------------------------------
+ * (3') Global-budget routing: the knapsack form of the error-aware routing
+ * (gist.science 2.B) taken over all blocks of a head at once.  Every block
+ * (a, c) with |q_a| > 0 and |k_c| > 0 costs |q_a| |k_c| pairs and is ranked
+ * by its unshifted error-to-cost ratio E[h][a][c] e^{2 M[h][a]}, compared as
+ * logf(E) + 2 M in float32 (E = 0 ranks last); equal keys: smaller a*Ck + c
+ * first.  The longest prefix whose total cost fits floor(rho * Nq * Nk)
+ * (exact integer arithmetic on the float32 rho) is routed.
+ *   E [H,Cq,Ck], M [H,Cq] from svgear_block_error (any router); the other
+ *   arguments and outputs as svgear_route.  sel lists each row's routed
+ *   clusters in that row's order; rows with |q_a| = 0 route nothing.
+ *   Ck <= 4096; Nq * Nk < 2^62 (else SVGEAR_ERR_UNSUPPORTED).
+ * ------------------------------------------------------------------------- */
+SVGEAR_API int svgear_route_global(const float* E, const float* M, const int32_t* k_counts,
+                        const int32_t* q_counts, const svgear_params* p, uint8_t* mask,
+                        int32_t* sel, int32_t* n_sel, int64_t* exec_pairs, void* stream);
+
+/* ---------------------------------------------------------------------------
  * (4) Hybrid attention.  Review step (4); gist.science 2.A "lineare
  * Kompensation".  For query i of cluster a (permuted order):
  *   o_i = sum over routed c, j in c of e^{s q_i.k_j} v_j
@@ -258,7 +284,8 @@ SVGEAR_API int svgear_hybrid_attn(const void* Qp, const void* Kp, const void* Vp
                        void* ws, size_t ws_bytes, void* stream);
 
 /* ---------------------------------------------------------------------------
- * The whole operator: (1) -> (1') -> (2) -> (3) -> (4) on one stream.
+ * The whole operator: (1) -> (1') -> (2) -> (3) -> (4) on one stream
+ * ((3') instead of (3) when p->budget is SVGEAR_BUDGET_GLOBAL).
  *   Q [H,Nq,d], K/V [H,Nk,d], O [H,Nq,d] in `dtype`.
  *   init_q [H,Cq,d] / init_k [H,Ck,d] float32 k-means initial centroids
  *   (NULL: deterministic init, see svgear_kmeans).

@@ -83,3 +83,10 @@ def test_validation_rejects_before_any_launch(L):
         assert sv.svgear_workspace_size(bad) == 0
     for r in (sv.SVGEAR_ROUTE_MASS, sv.SVGEAR_ROUTE_ERROR_NOV):
         assert sv.svgear_workspace_size(sv.params(1, 256, 256, 64, 4, 8, 2, 0.5, router=r)) > 0
+    # budget form outside svgear_budget
+    for b in (-1, 2):
+        bad = sv.params(1, 256, 256, 64, 4, 8, 2, 0.5, budget=b)
+        assert sv.svgear_workspace_size(bad) == 0
+    g = sv.params(1, 256, 256, 64, 4, 8, 2, 0.5, budget=sv.SVGEAR_BUDGET_GLOBAL)
+    assert sv.svgear_workspace_size(g) > 0
+    assert L.svgear_route_global(16, None, 16, 16, ctypes.byref(g), 16, 16, 16, 16, None) == sv.SVGEAR_ERR_INVALID

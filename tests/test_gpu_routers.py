@@ -1,7 +1,7 @@
-"""GPU parity of the two routing-signal ablations (attention mass and the
-value-agnostic error) against the oracle: the signal stage on the oracle's
-clusters, then whole forwards whose routing and output are checked against
-the oracle given the GPU's own upstream results."""
+"""GPU parity of the routing ablations against the oracle: the two ranking
+signals (attention mass and the value-agnostic error) on the oracle's clusters,
+global-budget routing on the oracle's errors, then whole forwards whose routing
+and output are checked against the oracle given the GPU's own upstream results."""
 import numpy as np
 import pytest
 
@@ -95,3 +95,82 @@ def test_forward_with_ablation_router(name, rho, router):
         # hybrid attention from the GPU's clusters and routing
         Oo = ora.hybrid_attention(cs.q[i], cs.k[i], cs.v[i], lq, lk, ck, vbar, kc, mask, cs.scale)
         assert_close(O[i], Oo, atol, rtol, f"{router} forward output head {i}")
+
+
+# ------------------------------------------------------------ global budget
+
+def _global_keys(E, M):
+    with np.errstate(divide="ignore"):
+        return np.log(np.maximum(np.asarray(E, np.float64), 0.0)) + 2.0 * np.asarray(M, np.float64)[:, None]
+
+
+def _check_global(mask, n_sel, sel, pairs, E, M, kc, qc, rho):
+    """GPU global routing against the oracle's from the same float32 E, M:
+    identical, or differing only on items whose keys are near-tied at the cut."""
+    mask_o, sel_o, pairs_o = ora.route_global(E, M, kc, qc, rho)
+    budget = ora.route_global_budget(rho, int(qc.sum()), int(kc.sum()))
+    cost = qc[:, None].astype(np.int64) * kc[None, :]
+    assert pairs == int((cost * mask).sum()) <= budget
+    assert (mask[qc == 0] == 0).all() and (mask[:, kc == 0] == 0).all()
+    diff = mask != mask_o
+    if diff.any():
+        key = _global_keys(E, M)[diff]
+        assert np.isfinite(key).all() and key.max() - key.min() <= 1e-5 * max(1.0, np.abs(key).max()), \
+            f"{diff.sum()} routing decisions differ away from the cut"
+    else:
+        assert pairs == pairs_o
+        for a in range(mask.shape[0]):
+            assert n_sel[a] == len(sel_o[a])
+            # the row's order; near-equal keys inside a row may swap
+            assert set(sel[a, :n_sel[a]]) == set(sel_o[a])
+
+
+@pytest.mark.parametrize("name,rho", [("tiny", None), ("mid", None), ("mid", 0.05), ("mid", 0.0), ("mid", 1.0)])
+def test_route_global_given_oracle_errors(name, rho):
+    cs = case(name, rho=rho)
+    cfg = cs.cfg
+    H, Cq, Ck = cs.H, cfg.Cq, cfg.Ck
+    E = np.stack([o["E"] for o in cs.oracle]).astype(np.float32)
+    M = np.stack([o["M"] for o in cs.oracle]).astype(np.float32)
+    kc = np.stack([o["k_counts"] for o in cs.oracle]).astype(np.int32)
+    qc = np.stack([o["q_counts"] for o in cs.oracle]).astype(np.int32)
+    # an empty query cluster routes nothing (members moved, total kept at N_q)
+    qc[0, 0] += qc[0, 1]
+    qc[0, 1] = 0
+    p = cs.params()
+    mask = torch.empty((H, Cq, Ck), dtype=torch.uint8, device="cuda")
+    sel = torch.empty((H, Cq, Ck), dtype=torch.int32, device="cuda")
+    n_sel = torch.empty((H, Cq), dtype=torch.int32, device="cuda")
+    pairs = torch.empty((H,), dtype=torch.int64, device="cuda")
+    sv.svgear_route_global(dev(E), dev(M), dev(kc), dev(qc), p, mask, sel, n_sel, pairs)
+    torch.cuda.synchronize()
+    mask, sel, n_sel, pairs = host(mask), host(sel), host(n_sel), host(pairs)
+    for i in range(H):
+        _check_global(mask[i], n_sel[i], sel[i], int(pairs[i]), E[i], M[i], kc[i].astype(np.int64),
+                      qc[i].astype(np.int64), cs.rho)
+    if cs.rho == 1.0:
+        assert (pairs == cfg.N * cfg.N).all()
+    if cs.rho == 0.0:
+        assert mask.sum() == 0
+
+
+@pytest.mark.parametrize("name,rho", [("tiny", None), ("mid", None), ("mid", 0.1)])
+def test_forward_with_global_budget(name, rho):
+    cs = case(name, rho=rho)
+    cfg = cs.cfg
+    O, ws, p, _ = sv.forward(cs.dq(), cs.dk(), cs.dv(), cfg.Cq, cfg.Ck, cfg.iters, cs.rho, cs.scale,
+                             dev(cs.init_q), dev(cs.init_k), budget=sv.SVGEAR_BUDGET_GLOBAL)
+    torch.cuda.synchronize()
+    assert sv.svgear_get_status() == sv.SVGEAR_OK
+    vw = sv.view_tensors(p, ws)
+    O = host(O)
+    atol, rtol = OUT_TOL[cfg.dtype]
+    for i in range(cs.H):
+        ck, vbar = (host(vw[n][i]).astype(np.float64) for n in ("cent_k", "vbar"))
+        lq, lk = host(vw["labels_q"][i]), host(vw["labels_k"][i])
+        kc, qc = host(vw["counts_k"][i]).astype(np.int64), host(vw["counts_q"][i]).astype(np.int64)
+        mask = host(vw["mask"][i])
+        _check_global(mask, host(vw["n_sel"][i]), host(vw["sel"][i]), int(host(vw["exec_pairs"][i])),
+                      host(vw["E"][i]), host(vw["M"][i]), kc, qc, cs.rho)
+        Oo = ora.hybrid_attention(cs.q[i], cs.k[i], cs.v[i], lq, lk, ck, vbar, kc, mask, cs.scale)
+        assert_close(O[i], Oo, atol, rtol, f"global-budget forward output head {i}")
