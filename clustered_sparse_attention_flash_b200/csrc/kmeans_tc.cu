@@ -24,6 +24,14 @@
 // 128-column chunks.  When a tile has chunks in both warpgroups, the one that
 // did not see the tile's last chunk hands its partial top three to the other
 // through shared memory (mbarrier-synchronised, no lockstep).
+//
+// When the bf16 centroids do not fit in shared memory next to two token
+// stages (d = 128 and more than 512 centroids), the centroids are taken in
+// segments of whole 128-column chunks, one launch per segment: every launch
+// but the last stores each token's top three (packed scores carry the global
+// column index) to a [3][H][N] buffer, every launch but the first folds the
+// stored top three in before its own decision or store, so the last launch
+// decides over all centroids with the same rule.
 #include <cuda.h>
 
 #include <algorithm>
@@ -400,7 +408,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const int2* __restrict__ table, const Bounds* __restrict__ bounds,
                 const float* __restrict__ xnorm, int N, int Cpad, int Cr, int stages, int tiles_per_cta,
                 int nbits, int32_t* __restrict__ labels, int4* __restrict__ list2,
-                int* __restrict__ list_full, int* __restrict__ counts, int* status) {
+                int* __restrict__ list_full, int* __restrict__ counts, int* status, int tstride, int c_base,
+                float* __restrict__ part, int pmode) {
+  // Cpad / Cr: padded columns / resident rows of this launch's centroid
+  // segment, which starts at global column c_base; tstride: the table's
+  // per-head stride.  pmode bit 0: fold in the top three stored by the
+  // previous segment; bit 1: store the top three instead of deciding.
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const Lay L = layout(D, Cr, Cpad, stages);
@@ -446,7 +459,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     *abort_flag = 0;
     tc::mbar_fence_init();
   }
-  for (int c = threadIdx.x; c < Cpad; c += blockDim.x) tab[c] = table[(size_t)h * Cpad + c];
+  for (int c = threadIdx.x; c < Cpad; c += blockDim.x) tab[c] = table[(size_t)h * tstride + c_base + c];
   if (warp == 0) {
     tc::tmem_alloc(tmem_slot, 512);
     tc::tmem_relinquish();
@@ -499,8 +512,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc::mbar_arrive_expect_tx(cent_full, (uint32_t)(Cr * D * 2));
       for (int kh = 0; kh < D / 64; ++kh)
         for (int rb = 0; rb < Cr / 128; ++rb)
-          tc::tma_load_3d(cent_a + (uint32_t)(kh * Cr * 128 + rb * 128 * 128), &tmc, kh * 64, rb * 128, h,
-                          cent_full);
+          tc::tma_load_3d(cent_a + (uint32_t)(kh * Cr * 128 + rb * 128 * 128), &tmc, kh * 64, c_base + rb * 128,
+                          h, cent_full);
       for (int t = 0; t < nt; ++t) {
         const int s = t % stages, k = t / stages;
         if (!tc::mbar_wait(x_empty + s, (k & 1) ^ 1, abort_flag, status)) break;
@@ -588,6 +601,21 @@ __global__ void __launch_bounds__(kThreads, 1)
         b3 = n3;
       }
       const int row = (t0 + t) * BM + r;
+      if (pmode != 0) {
+        const size_t plane = (size_t)gridDim.y * N, at = (size_t)h * N + row;
+        if ((pmode & 1) && row < N) {  // the previous segments' top three
+          const float c1 = part[at], c2 = part[plane + at], c3 = part[2 * plane + at];
+          const float n3 = fmaxf(tc::fmax3(b3, fminf(b2, c1), fminf(b1, c2)), c3);
+          const float n2 = tc::fmax3(b2, fminf(b1, c1), c2);
+          b1 = fmaxf(b1, c1);
+          b2 = n2;
+          b3 = n3;
+        }
+        if (pmode & 2) {  // a later segment decides (pmode is uniform)
+          if (row < N) { part[at] = b1; part[plane + at] = b2; part[2 * plane + at] = b3; }
+          continue;
+        }
+      }
       int need = 0, lab = 0;
       if (row < N) {
         const float xn = xnorm[(size_t)h * N + row];
@@ -629,17 +657,29 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 }  // namespace
 
-static int pick_stages(int d, int C) {
-  const int Cpad = round16(C), Cr = round128(C);
+// Token stages that fit next to a centroid segment of Cpad columns (Cr rows).
+static int pick_stages(int d, int Cr, int Cpad) {
   int s = 0;
   while (s < kMaxStages && layout(d, Cr, Cpad, s + 1).total <= kSmemLimit) ++s;
   return s;
 }
 
+// Columns per launch: all of them (round128(C)) when they fit with two token
+// stages, else the largest multiple of 128 that does (0: none).
+static int segment_cols(int d, int C) {
+  const int Cpad = round16(C), Cr = round128(C);
+  if (pick_stages(d, Cr, Cpad) >= 2) return Cr;
+  int s = Cr - kChunk;
+  while (s >= kChunk && pick_stages(d, s, s) < 2) s -= kChunk;
+  return s;
+}
+
+static bool segmented(int d, int C) { return segment_cols(d, C) < round16(C); }
+
 bool kmeans_tc_supported(int d, int C) {
   if (d != 64 && d != 128) return false;
   if (C < 1 || C > kMaxC) return false;
-  return pick_stages(d, C) >= 2;
+  return segment_cols(d, C) >= kChunk;
 }
 
 bool kmeans_tc_usable(const void* X, int N, int d, int C) {
@@ -660,6 +700,7 @@ struct TcWs {
   int* counts;  // [0] two-candidate rows, [1 + h] full-scan rows of head h
   int4* list2;
   int* list_full;  // [H][N]
+  float* part;     // [3][H][N] top three between centroid segments (segmented shapes only)
 };
 
 static size_t zeroed_bytes(int H) { return sizeof(Bounds) * H + sizeof(int) * ((size_t)H + 1); }
@@ -677,6 +718,7 @@ static size_t tc_layout(int H, int N, int d, int C, TcWs* out, void* ws) {
   w.counts = z ? reinterpret_cast<int*>(z + sizeof(Bounds) * H) : nullptr;
   w.list2 = cv.take<int4>((size_t)H * N);
   w.list_full = cv.take<int>((size_t)H * N);
+  w.part = segmented(d, C) ? cv.take<float>((size_t)3 * H * N) : nullptr;
   if (out) *out = w;
   return cv.used();
 }
@@ -714,7 +756,8 @@ template <int D>
 static cudaError_t assign_launch(const bf16* X, int H, int N, int C, const float* cent, int32_t* labels,
                                  const TcWs& w, cudaStream_t st) {
   const int Cpad = round16(C), Cr = round128(C);
-  const int stages = pick_stages(D, C);
+  const int seg = segment_cols(D, C);
+  if (seg < kChunk || (seg < Cpad && !w.part)) return cudaErrorInvalidValue;
   int nbits = 1;
   while ((1 << nbits) < Cpad) ++nbits;
   k_prep_centroids<D><<<dim3(Cr / 32, H), 256, 0, st>>>(cent, C, Cpad, Cr, w.cb, w.table, w.centT, w.bd);
@@ -722,15 +765,20 @@ static cudaError_t assign_launch(const bf16* X, int H, int N, int C, const float
   CUtensorMap tmx, tmc;
   if (!tma_map_bf16_3d(&tmx, X, D, N, H, BM) || !tma_map_bf16_3d(&tmc, w.cb, D, Cr, H, 128))
     return cudaErrorInvalidValue;
-  const int smem = layout(D, Cr, Cpad, stages).total;
-  cudaError_t e = cudaFuncSetAttribute(k_assign_tc<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-  if (e != cudaSuccess) return e;
   const int T = (N + BM - 1) / BM;
   const int tpc = pick_tiles_per_cta(H, T);
-  k_assign_tc<D><<<dim3((T + tpc - 1) / tpc, H), kThreads, smem, st>>>(
-      tmx, tmc, w.table, w.bd, w.xn, N, Cpad, Cr, stages, tpc, nbits, labels, w.list2, w.list_full,
-      w.counts, status_word());
-  note_launch();
+  for (int c_base = 0; c_base < Cpad; c_base += seg) {
+    const int sp = std::min(seg, Cpad - c_base), sr = round128(sp);
+    const int stages = pick_stages(D, sr, sp);
+    const int pmode = (c_base > 0 ? 1 : 0) | (c_base + seg < Cpad ? 2 : 0);
+    const int smem = layout(D, sr, sp, stages).total;
+    cudaError_t e = cudaFuncSetAttribute(k_assign_tc<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    k_assign_tc<D><<<dim3((T + tpc - 1) / tpc, H), kThreads, smem, st>>>(
+        tmx, tmc, w.table, w.bd, w.xn, N, sp, sr, stages, tpc, nbits, labels, w.list2, w.list_full,
+        w.counts, status_word(), Cpad, c_base, w.part, pmode);
+    note_launch();
+  }
   k_refine2<D><<<148 * 4, 256, 0, st>>>(X, cent, N, C, w.list2, w.counts, labels);
   note_launch();
   const int fthreads = C > kFullThreads ? kFullThreads : (C + 31) / 32 * 32;

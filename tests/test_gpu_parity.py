@@ -331,6 +331,9 @@ def test_forward_empty_key_cluster():
     (20000, 128, 300, 1),    # second slot ends in a 16-column tail
     (9001, 64, 1000, 2),     # d = 64: four slots alternate between warpgroups
     (5000, 128, 100, 3),     # one slot, tiles alternate between warpgroups
+    (30000, 128, 1000, 4),   # centroids in two segments of 512 columns (HunyuanVideo-shaped keys)
+    (9001, 128, 700, 5),     # segments of 512 and 192 columns
+    (5000, 128, 513, 6),     # second segment is one 16-column chunk
 ])
 def test_kmeans_assign_wide(N, d, C, seed):
     from clustered_sparse_attention_flash_b200.synth import to_bf16_f32
