@@ -36,6 +36,11 @@ Readings taken where the pages are silent (each listed in the design notes):
 * Hybrid attention: every compensated key cluster contributes |k_c| copies of
   its centroid term, i.e. a logit bias log|k_c|, inside the same softmax as the
   exact keys (one maximum, one normaliser).
+* Ablations (not the method; they swap one ingredient of the routing): a
+  score-based signal, the attention weight |k_c| e^{s qbar.kbar_c} the query
+  centroid gives each key cluster, normalised per row; the block error without
+  the values; one budget of floor(rho N_q N_k) pairs per head over all blocks,
+  ranked by the unshifted ratio.
 
 Arrays are per head: X [N, d]; centroids [C, d]; labels [N] ints.
 """
