@@ -1,0 +1,57 @@
+"""bench.py's host-side helpers, no GPU: the DRAM-traffic figure is reported
+only for the workload and kernel sources it was captured on, the stress
+sweep's trend test, the workload description and the generator's
+configuration override."""
+import hashlib
+import os
+
+import numpy as np
+import pytest
+
+import bench
+from clustered_sparse_attention_flash_b200 import synth
+
+
+def _sources_hash():
+    h = hashlib.sha1()
+    for f in bench._ATTN_TRAFFIC["sources"]:
+        with open(os.path.join(bench.ROOT, "clustered_sparse_attention_flash_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()
+
+
+def test_attention_traffic_only_for_its_capture():
+    wan = synth.CONFIGS["wan"]
+    assert bench.attn_traffic(synth.CONFIGS["stress"]) is None
+    t = bench.attn_traffic(wan)
+    if _sources_hash() == bench._ATTN_TRAFFIC["sha1"]:
+        assert t == pytest.approx(bench._ATTN_TRAFFIC["bytes_per_head"] * wan.H)
+        assert bench.attn_traffic(wan.with_(H=4)) == pytest.approx(324.9e6)
+    else:
+        assert t is None
+
+
+def test_trend_helper():
+    assert bench._nonincreasing([3.0, 2.0, 2.0, 1.0])
+    assert not bench._nonincreasing([1.0, 2.0])
+    assert bench._nonincreasing([])
+    assert bench._nonincreasing([1.0, 1.0 + 1e-9], slack=1.0 + 1e-6)
+
+
+def test_workload_names_sizes():
+    w = bench._workload(synth.CONFIGS["wan"], 0.15)
+    for part in ("H=40", "N=75600", "21x45x80", "d=128", "Cq=100", "Ck=500", "rho=0.15"):
+        assert part in w
+
+
+def test_generator_honours_the_config_it_is_given():
+    """The stress sweep overrides sigma; each head must be generated from the
+    overridden configuration, not the registered one."""
+    base = synth.CONFIGS["tiny"]
+    a = bench._gen_head((base.with_(sigma=0.1), 0))
+    b = bench._gen_head((base.with_(sigma=1.0), 0))
+    c = bench._gen_head((base.with_(sigma=1.0), 0))
+    assert not np.array_equal(a[0], b[0])
+    for x, y in zip(b, c):
+        np.testing.assert_array_equal(x, y)
+    assert a[3].shape == (base.Cq, base.d) and a[4].shape == (base.Ck, base.d)
