@@ -434,6 +434,23 @@ def test_route_global_depends_on_unshifted_ratio_only():
         assert a[2] == b[2] <= ora.route_global_budget(rho, qc.sum(), kc.sum())
 
 
+def test_route_global_one_query_cluster_is_row_routing():
+    """With a single query cluster the pair budget floor(rho N_q N_k) over
+    costs N_q |k_c| is the key budget floor(rho N_k), and the global order is
+    the row's order: the two routings coincide."""
+    rng = np.random.default_rng(33)
+    for trial in range(20):
+        Ck = int(rng.integers(1, 40))
+        E = rng.random((1, Ck)) ** 2
+        kc = rng.integers(0, 7, Ck); kc[rng.integers(Ck)] += 1
+        qc = np.array([int(rng.integers(1, 50))])
+        rho = float(rng.random())
+        mg, sg, pg = ora.route_global(E, rng.normal(size=1), kc, qc, rho)
+        mr, sr, pr = ora.route(E, kc, qc, rho)
+        np.testing.assert_array_equal(mg, mr)
+        assert list(sg[0]) == list(sr[0]) and pg == pr
+
+
 def test_route_global_extremes():
     rng = np.random.default_rng(32)
     E = rng.random((4, 6)); M = rng.normal(size=4)
