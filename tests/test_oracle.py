@@ -411,6 +411,15 @@ def test_route_global_worked_example():
     assert not np.array_equal(m2, mask)
 
 
+def test_route_global_equal_ratios_go_to_the_smaller_block_index():
+    """Four blocks of one pair each with the same ratio and a budget of two
+    pairs: the blocks (0,0) and (0,1), first in a*Ck + c order, are routed."""
+    E = np.full((2, 2), 0.5)
+    mask, sel, pairs = ora.route_global(E, np.zeros(2), np.array([1, 1]), np.array([1, 1]), 0.5)
+    np.testing.assert_array_equal(mask, [[1, 1], [0, 0]])
+    assert pairs == 2 and [list(x) for x in sel] == [[0, 1], []]
+
+
 def test_route_global_budget_is_exact():
     """float32(0.1) = 0.100000001490116119384765625; times 75,600^2 =
     5,715,360,000 gives 571,536,008.5166..., floor 571,536,008."""
