@@ -61,6 +61,10 @@ constexpr int kUnitRows = BQ;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr uint32_t kColS = 0, kColO = 256;
 constexpr int kMaxRanges = 512;  // routed clusters staged in shared memory
+constexpr int kRegsLow = 56;     // MMA / producer warpgroup after the split
+constexpr int kRegsHigh = 208;   // each softmax warpgroup after the split
+// the split fits a launch of 168 registers per thread (checked at launch)
+static_assert(4 * 32 * kRegsLow + 8 * 32 * kRegsHigh <= kThreads * 168, "register split");
 
 __device__ __forceinline__ float ex2(float x) {
   float y;
@@ -350,6 +354,14 @@ __global__ void __launch_bounds__(kThreads, 1)
   auto ustart = [&](int j) { return j <= n_ex ? j : n_ex + 2 * (j - n_ex); };
   auto nparts = [&](int j) { return j < n_ex ? 1 : 2; };
 
+  // Register split between the warpgroups: the MMA / producer warpgroup
+  // gives registers back, the two softmax warpgroups take them (one S row of
+  // 128 values stays in registers).  4 warps x 32 x kRegsLow + 8 warps x 32 x
+  // kRegsHigh must not exceed the block's registers at launch (384 threads
+  // x the compiled count, checked on the host before the first launch).
+  if (warp < 4) tc::setmaxnreg_dec<kRegsLow>();
+  else tc::setmaxnreg_inc<kRegsHigh>();
+
   if (warp == 0) {
     // ------------------------------------------------------------------ MMA
     if (lane == 0) {
@@ -615,31 +627,33 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!tc::mbar_wait_warp(v_full + st, (u0 / kVSlots) & 1, abort_flag, status)) { ok = false; break; }
       tc::tc_fence_after();
       const float* bias = bias_s + st * BN;
-      // pass 1: the row maximum over the stage's 128 keys, 64 at a time
-      float mx = -INFINITY;
-#pragma unroll 1
-      for (int h2 = 0; h2 < 2; ++h2) {
-        uint32_t v[64];
-        tc::tmem_ld32(tmem + lane_base + scol + (uint32_t)(h2 * 64), *reinterpret_cast<uint32_t(*)[32]>(v));
-        tc::tmem_ld32(tmem + lane_base + scol + (uint32_t)(h2 * 64 + 32), *reinterpret_cast<uint32_t(*)[32]>(v + 32));
-        tc::tmem_ld_wait();
+      // the stage's 128 logits of this row, read once: x = s*log2e * S + bias
+      uint32_t v[128];
+      tc::tmem_ld32(tmem + lane_base + scol, *reinterpret_cast<uint32_t(*)[32]>(v));
+      tc::tmem_ld32(tmem + lane_base + scol + 32u, *reinterpret_cast<uint32_t(*)[32]>(v + 32));
+      tc::tmem_ld32(tmem + lane_base + scol + 64u, *reinterpret_cast<uint32_t(*)[32]>(v + 64));
+      tc::tmem_ld32(tmem + lane_base + scol + 96u, *reinterpret_cast<uint32_t(*)[32]>(v + 96));
+      tc::tmem_ld_wait();
+      float mx;
+      {
         float m8[8];
 #pragma unroll
         for (int k = 0; k < 8; ++k) m8[k] = -INFINITY;
 #pragma unroll
-        for (int i = 0; i < 64; i += 16) {
-          const float4 b0 = *reinterpret_cast<const float4*>(bias + h2 * 64 + i);
-          const float4 b1 = *reinterpret_cast<const float4*>(bias + h2 * 64 + i + 4);
-          const float4 b2 = *reinterpret_cast<const float4*>(bias + h2 * 64 + i + 8);
-          const float4 b3 = *reinterpret_cast<const float4*>(bias + h2 * 64 + i + 12);
+        for (int i = 0; i < 128; i += 16) {
+          const float4 b0 = *reinterpret_cast<const float4*>(bias + i);
+          const float4 b1 = *reinterpret_cast<const float4*>(bias + i + 4);
+          const float4 b2 = *reinterpret_cast<const float4*>(bias + i + 8);
+          const float4 b3 = *reinterpret_cast<const float4*>(bias + i + 12);
           const float bb[16] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w,
                                 b2.x, b2.y, b2.z, b2.w, b3.x, b3.y, b3.z, b3.w};
 #pragma unroll
+          for (int k = 0; k < 16; ++k) v[i + k] = __float_as_uint(fmaf(__uint_as_float(v[i + k]), scale2, bb[k]));
+#pragma unroll
           for (int k = 0; k < 8; ++k)
-            m8[k] = tc::fmax3(m8[k], fmaf(__uint_as_float(v[i + k]), scale2, bb[k]),
-                              fmaf(__uint_as_float(v[i + 8 + k]), scale2, bb[8 + k]));
+            m8[k] = tc::fmax3(m8[k], __uint_as_float(v[i + k]), __uint_as_float(v[i + 8 + k]));
         }
-        mx = fmaxf(mx, fmaxf(tc::fmax3(m8[0], m8[1], m8[2]), tc::fmax3(tc::fmax3(m8[3], m8[4], m8[5]), m8[6], m8[7])));
+        mx = fmaxf(tc::fmax3(m8[0], m8[1], m8[2]), tc::fmax3(tc::fmax3(m8[3], m8[4], m8[5]), m8[6], m8[7]));
       }
       // lazy rescale: a row whose maximum grew by more than 2^8 rescales O[w]
       // and l_w.  The tensor-memory accesses are warp-collective, so the warp
@@ -664,33 +678,21 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       if (grow) m_used = mx;
       const float mref = m_used == -INFINITY ? 0.f : m_used;
-      // pass 2: P = 2^(x - m) in bf16 over the first 64 columns of S[w]
-      // (keys 64 h2 + [0, 64) in columns 32 h2 + [0, 32), after they are read)
+      // P = 2^(x - m) in bf16 over the first 64 columns of S[w] (keys 2c and
+      // 2c + 1 in column c; every S value of the row is already in registers)
       float r8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-#pragma unroll 1
-      for (int h2 = 0; h2 < 2; ++h2) {
-        uint32_t v[64];
-        tc::tmem_ld32(tmem + lane_base + scol + (uint32_t)(h2 * 64), *reinterpret_cast<uint32_t(*)[32]>(v));
-        tc::tmem_ld32(tmem + lane_base + scol + (uint32_t)(h2 * 64 + 32), *reinterpret_cast<uint32_t(*)[32]>(v + 32));
-        tc::tmem_ld_wait();
 #pragma unroll
-        for (int q = 0; q < 2; ++q) {
-          uint32_t pk[16];
+      for (int q = 0; q < 4; ++q) {
+        uint32_t pk[16];
 #pragma unroll
-          for (int i = 0; i < 16; i += 2) {
-            const float4 b4 = *reinterpret_cast<const float4*>(bias + h2 * 64 + q * 32 + 2 * i);
-            const int c = q * 32 + 2 * i;
-            const float p0 = ex2(fmaf(__uint_as_float(v[c]), scale2, b4.x) - mref);
-            const float p1 = ex2(fmaf(__uint_as_float(v[c + 1]), scale2, b4.y) - mref);
-            const float p2 = ex2(fmaf(__uint_as_float(v[c + 2]), scale2, b4.z) - mref);
-            const float p3 = ex2(fmaf(__uint_as_float(v[c + 3]), scale2, b4.w) - mref);
-            r8[i & 7] += p0 + p1;
-            r8[(i + 1) & 7] += p2 + p3;
-            pk[i] = pack_bf16(p0, p1);
-            pk[i + 1] = pack_bf16(p2, p3);
-          }
-          tc::tmem_st16(tmem + lane_base + scol + (uint32_t)(h2 * 32 + q * 16), pk);
+        for (int i = 0; i < 16; ++i) {
+          const int c = q * 32 + 2 * i;
+          const float p0 = ex2(__uint_as_float(v[c]) - mref);
+          const float p1 = ex2(__uint_as_float(v[c + 1]) - mref);
+          r8[i & 7] += p0 + p1;
+          pk[i] = pack_bf16(p0, p1);
         }
+        tc::tmem_st16(tmem + lane_base + scol + (uint32_t)(q * 16), pk);
       }
       tc::tmem_st_wait();
       l += ((r8[0] + r8[1]) + (r8[2] + r8[3])) + ((r8[4] + r8[5]) + (r8[6] + r8[7]));
@@ -808,6 +810,12 @@ cudaError_t launch(const void* Qp, const void* Kp, const void* Vp, const int32_t
   const int smem = AttnSmem<D>::total;
   cudaError_t e = cudaFuncSetAttribute(k_attn_tc<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
+  // the softmax warpgroups' register increase waits for the pool the block
+  // was launched with: refuse a build whose launch count cannot cover it
+  cudaFuncAttributes fa;
+  e = cudaFuncGetAttributes(&fa, k_attn_tc<D>);
+  if (e != cudaSuccess) return e;
+  if ((long long)fa.numRegs * kThreads < 4LL * 32 * kRegsLow + 8LL * 32 * kRegsHigh) return cudaErrorInvalidValue;
   k_attn_tc<D><<<dim3(tmax, H), kThreads, smem, st>>>(
       static_cast<const bf16*>(Qp), w.kpk, w.vpk, w.npad, q_off, k_off, w.poff, perm_q, w.kh, w.kl, w.vh, w.vl,
       w.lc2, sel, n_sel, w.tiles, w.ntiles, tmax, Nq, Nk, Cq, Ck, Ckpad, scale * kLog2e,
