@@ -41,7 +41,23 @@ __global__ void __launch_bounds__(256) k_value_stats(const T* __restrict__ Vp, c
   double acc[PER];
 #pragma unroll
   for (int t = 0; t < PER; ++t) acc[t] = 0.0;
-  for (int r = beg + w; r < end; r += NW) {
+  int r0 = beg + w;
+  for (; r0 + 3 * NW < end; r0 += 4 * NW) {  // four rows in flight per warp
+    if constexpr (PER == 4) {
+      float4 v[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) v[u] = ld4(Vh + (size_t)(r0 + u * NW) * D);
+#pragma unroll
+      for (int u = 0; u < 4; ++u) { acc[0] += v[u].x; acc[1] += v[u].y; acc[2] += v[u].z; acc[3] += v[u].w; }
+    } else {
+      float2 v[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) v[u] = ld2(Vh + (size_t)(r0 + u * NW) * D);
+#pragma unroll
+      for (int u = 0; u < 4; ++u) { acc[0] += v[u].x; acc[1] += v[u].y; }
+    }
+  }
+  for (int r = r0; r < end; r += NW) {
     if constexpr (PER == 4) {
       float4 v = ld4(Vh + (size_t)r * D);
       acc[0] += v.x; acc[1] += v.y; acc[2] += v.z; acc[3] += v.w;
