@@ -126,6 +126,74 @@ def test_value_centroid_of_singleton_is_the_value():
 
 # ------------------------------------------------------------- block error ----
 
+def test_key_scalars_two_key_worked_example():
+    """Values (1, 0) and (3, 2) in one cluster: vbar = (2, 1).  Key 0:
+    vbar - v = (1, 1), so (2, 1, 1); key 1: vbar - v = (-1, -1), so
+    (2, -5, 13).  Worked by hand."""
+    V = np.array([[1.0, 0.0], [3.0, 2.0]])
+    lab = np.array([0, 0])
+    Vbar = np.array([[2.0, 1.0]])
+    np.testing.assert_array_equal(ora.key_scalars(V, lab, Vbar),
+                                  [[2.0, 2.0], [1.0, -5.0], [1.0, 13.0]])
+
+
+def test_key_scalars_reproduce_the_literal_error_norm():
+    """The block error's per-key term ||A vbar - B v||^2 equals
+    A^2 (s1 + 2 w s2 + w^2 s3) with w = (A - B) / A, because
+    A vbar - B v = A ((vbar - v) + w v).  Checked against the literal norm on
+    random values, weights and clusters; and the cross term summed over a
+    cluster is minus the summed squared deviation (sum_j (vbar - v_j).v_j =
+    n ||vbar||^2 - sum_j ||v_j||^2)."""
+    rng = np.random.default_rng(41)
+    V = rng.standard_normal((50, 6))
+    lab = rng.integers(0, 5, size=50)
+    Vbar = ora.value_centroids(V, lab, 5)
+    s1, s2, s3 = ora.key_scalars(V, lab, Vbar)
+    A = np.exp(rng.standard_normal(50))
+    B = np.exp(rng.standard_normal(50))
+    w = (A - B) / A
+    lit = ((A[:, None] * Vbar[lab] - B[:, None] * V) ** 2).sum(1)
+    np.testing.assert_allclose(A * A * (s1 + 2 * w * s2 + w * w * s3), lit, rtol=1e-12)
+    for c in range(5):
+        m = lab == c
+        assert s2[m].sum() == pytest.approx(-s1[m].sum(), rel=1e-12, abs=1e-12)
+        assert s1[m].sum() == pytest.approx(m.sum() * np.var(V[m], axis=0).sum(), rel=1e-12)
+
+
+def test_block_error_scale_worked_example():
+    """d = 1, qbar = 1, scale 1, keys {0, ln 2} (kbar = ln2 / 2), values
+    (1, 0) and (0, 2) with vbar = (1/2, 1): M = ln2 / 2, A = 1,
+    B = {2^-1/2, 2^1/2}, ||vbar||^2 = 5/4, ||v||^2 = {1, 4}, so
+    T = (1/2) ((5/4 + 1/2) + (5/4 + 8)) = 11/2.  Worked by hand."""
+    ln2 = math.log(2.0)
+    K = np.array([[0.0], [ln2]])
+    V = np.array([[1.0, 0.0], [0.0, 2.0]])
+    T = ora.block_error_scale(np.array([[1.0]]), np.array([[ln2 / 2]]), np.array([[0.5, 1.0]]),
+                              K, V, np.array([0, 0]), np.array([2]), 1.0)
+    assert T[0, 0] == pytest.approx(5.5, rel=1e-13)
+
+
+def test_block_error_scale_bounds_the_error():
+    """||a - b||^2 <= 2 (||a||^2 + ||b||^2) term by term, so E <= 2 T; with
+    values of zero mean in every cluster (vbar = 0) the cross term vanishes
+    and E = T exactly."""
+    rng = np.random.default_rng(42)
+    Qb = rng.standard_normal((3, 4))
+    K = rng.standard_normal((40, 4))
+    V = rng.standard_normal((40, 5))
+    lab = rng.integers(0, 6, size=40)
+    cnt = np.bincount(lab, minlength=6)
+    Kb = ora.value_centroids(K, lab, 6)
+    Vb = ora.value_centroids(V, lab, 6)
+    E, _ = ora.block_error(Qb, Kb, Vb, K, V, lab, cnt, 0.6)
+    T = ora.block_error_scale(Qb, Kb, Vb, K, V, lab, cnt, 0.6)
+    assert (E <= 2 * T * (1 + 1e-12)).all()
+    V0 = V - Vb[lab]  # zero mean per cluster
+    E0, _ = ora.block_error(Qb, Kb, np.zeros_like(Vb), K, V0, lab, cnt, 0.6)
+    T0 = ora.block_error_scale(Qb, Kb, np.zeros_like(Vb), K, V0, lab, cnt, 0.6)
+    np.testing.assert_allclose(E0, T0, rtol=1e-12, atol=1e-300)
+
+
 def test_block_error_zero_query_centroid_is_value_variance():
     """qbar = 0 makes every logit 0: A = B = 1, so E[a, c] is the
     within-cluster (population) variance of V, summed over dims."""
