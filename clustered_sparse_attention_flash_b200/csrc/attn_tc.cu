@@ -6,8 +6,9 @@
 //       / [ the same without v ],
 // written to row perm_q[i] of the output.
 //
-// One block per 128-row query tile of one query cluster (tiles never straddle
-// clusters, so a tile has one key stream):
+// One block per pair of 128-row query tiles of one query cluster (256
+// consecutive rows of the cluster; tiles never straddle clusters, so both
+// tiles share one key stream and every key / value stage is used by both):
 //   * exact part: the rows of the routed clusters (routing order),
 //     concatenated and cut into 128-key tiles (the last one masked),
 //   * compensation part: all key centroids in 128-row tiles, logit bias
@@ -19,27 +20,31 @@
 // padded to a multiple of 8 rows, each group of 8 rows stored as
 // [16-byte chunk][row]), which is directly a no-swizzle UMMA operand (K-major
 // for K, MN-major for V); a stage is one or a few contiguous runs, each moved
-// by a single cp.async.bulk.  K has a three-slot ring and V (with the stage's
-// bias vector) a two-slot ring: a K slot is free once S of its stage is
-// computed, a V slot once P.V is; padding rows are masked through the bias.
+// by a single cp.async.bulk.  K (with the stage's bias vector) and V each have
+// a two-slot ring: a K slot is free once S of its stage is computed for both
+// query tiles and both softmax groups have read the bias, a V slot once P.V is
+// done for both tiles; padding rows are masked through the bias.  A softmax
+// stage waits only for its S (and the bias that came with the keys), never for
+// the values, which load while it runs.  Sharing each stage between two query
+// tiles halves the key / value traffic from L2 per FLOP, which is what bounds
+// a one-tile block.
 // Warp roles (12 warps):
-//   warp 0      tensor-memory allocation, MMA issue (one thread): S = Q K^T
-//               into double-buffered S (N = 128 keys), then O[j % 2] += P V of
-//               the previous stage with P read from tensor memory;
-//   warps 1-3   load the query tile; warps 1 and 2 then produce the even
-//               and the odd stages (bulk copies issued by one lane, bias
+//   warp 0      tensor-memory allocation, MMA issue (one thread) in the order
+//               P.V_0(j), S_0(j+1), P.V_1(j), S_1(j+1): while the tensor core
+//               works for one query tile the other tile's softmax runs;
+//   warps 1-3   load the two query tiles; warps 1 and 2 then produce the
+//               even and the odd stages (bulk copies issued by one lane, bias
 //               vectors by the warp);
-//   warps 4-7   softmax of the even stages, warps 8-11 of the odd stages
-//               (thread = query row, all 128 keys of its stage): each group
-//               keeps its own running maximum, row sum and accumulator O[w],
-//               rescales O[w] lazily when its maximum grows by more than 2^8,
-//               writes P = 2^(x - m) in bf16 over the S columns of the stage;
-//               at the end the two partial results are merged (split-K style)
-//               and O / l is stored through perm_q.
-// Tensor memory (512 columns): S[0..1] [0,256), O[0..1] [256,256+2d); P[b]
-// lives in the first 64 columns of S[b].  Every decision that guards a
-// warp-collective tensor-memory access is made warp-uniform, and every wait
-// is time-bounded (device status word on expiry).
+//   warps 4-7   softmax of query tile 0, warps 8-11 of query tile 1 (thread =
+//               query row, all 128 keys of each stage): running maximum, row
+//               sum, lazy rescale of the tile's accumulator O[t] when the
+//               maximum grows by more than 2^8, P = 2^(x - m) in bf16 over the
+//               S columns of the tile; at the end O / l is stored through
+//               perm_q.
+// Tensor memory (512 columns): S[t] [128 t, 128 t + 128), O[t]
+// [256 + d t, 256 + d t + d); P[t] lives in the first 64 columns of S[t].
+// Every decision that guards a warp-collective tensor-memory access is made
+// warp-uniform, and every wait is time-bounded (device status word on expiry).
 #include <algorithm>
 #include <cmath>
 
@@ -51,13 +56,13 @@ namespace svg {
 
 namespace {
 
-constexpr int BQ = 128;        // rows per query tile (one tile per block)
+constexpr int BQ = 128;        // rows per query tile (two tiles per block)
 constexpr int BN = 128;        // keys per ring stage
 constexpr int kThreads = 384;
 constexpr int kProducers = 96;
-constexpr int kKSlots = 3;     // K ring (keys are needed first)
-constexpr int kVSlots = 2;     // V ring (with the stage's bias vector)
-constexpr int kUnitRows = BQ;
+constexpr int kKSlots = 2;     // K ring, with the stage's bias vector
+constexpr int kVSlots = 2;     // V ring
+constexpr int kUnitRows = 2 * BQ;  // query rows of one block
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr uint32_t kColS = 0, kColO = 256;
 constexpr int kMaxRanges = 512;  // routed clusters staged in shared memory
@@ -217,16 +222,13 @@ __global__ void k_tile_table_tc(const int32_t* __restrict__ q_off, int Cq, int t
 
 template <int D>
 struct AttnSmem {
-  static constexpr int kQTile = BQ * D * 2;   // the 128-row bf16 query tile
+  static constexpr int kQTile = BQ * D * 2;   // one 128-row bf16 query tile
   static constexpr int kKTile = BN * D * 2;   // one 128-row bf16 key (or value) tile
-  static constexpr int q_off = 0;
-  static constexpr int k_off = q_off + kQTile;                       // [kKSlots] key tiles
+  static constexpr int q_off = 0;                                    // [2] query tiles
+  static constexpr int k_off = q_off + 2 * kQTile;                   // [kKSlots] key tiles
   static constexpr int v_off = k_off + kKSlots * kKTile;             // [kVSlots] value tiles
-  static constexpr int bias_off = v_off + kVSlots * kKTile;          // [kVSlots][BN] log2 biases
-  static constexpr int mx_off = bias_off + kVSlots * BN * 4;         // [2 groups][BQ] row maxima
-  static constexpr int ls_off = mx_off + 2 * 2 * BQ * 4;             // [2 groups][BQ] row sums
-  static constexpr int flag_off = ls_off + 2 * BQ * 4;               // [kVSlots]: 1 = apply bias
-  static constexpr int bits_off = flag_off + 64;
+  static constexpr int bias_off = v_off + kVSlots * kKTile;          // [kKSlots][BN] log2 biases
+  static constexpr int bits_off = bias_off + kKSlots * BN * 4;
   static constexpr int rng_off = bits_off + kMaxCkBits / 8;          // [3][kMaxRanges] start, prefix, len
   static constexpr int pc_off = rng_off + 3 * kMaxRanges * 4 + 16;   // [producer warp][32] piece lists
   static constexpr int bar_off = pc_off + 2 * 32 * 16;
@@ -255,9 +257,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   float* bias_s = reinterpret_cast<float*>(smem + S::bias_off);
-  float* mx_s = reinterpret_cast<float*>(smem + S::mx_off);
-  float* ls_s = reinterpret_cast<float*>(smem + S::ls_off);
-  int* flag_s = reinterpret_cast<int*>(smem + S::flag_off);
   uint32_t* bits = reinterpret_cast<uint32_t*>(smem + S::bits_off);
   int* rng_start = reinterpret_cast<int*>(smem + S::rng_off);  // first padded row of routed range i
   int* rng_cum = rng_start + kMaxRanges;                        // padded rows in ranges [0, i)
@@ -266,13 +265,12 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + S::bar_off);
   uint64_t* q_full = bars + 0;
   uint64_t* k_full = bars + 1;     // [kKSlots]
-  uint64_t* k_empty = bars + 4;    // [kKSlots]
+  uint64_t* k_empty = bars + 4;    // [kKSlots]: S of the stage done + its bias read by every softmax warp
   uint64_t* v_full = bars + 7;     // [kVSlots]
   uint64_t* v_empty = bars + 9;    // [kVSlots]
-  uint64_t* s_full = bars + 11;    // [2]
-  uint64_t* p_full = bars + 13;    // [2]
-  uint64_t* o_done = bars + 15;    // [2]
-  uint64_t* l_bar = bars + 17;     // both softmax groups posted their row maxima and sums
+  uint64_t* s_full = bars + 11;    // [2 query tiles]
+  uint64_t* p_full = bars + 13;    // [2 query tiles]
+  uint64_t* o_done = bars + 15;    // [2 query tiles]
   uint64_t* done = bars + 18;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 19);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 20);
@@ -280,6 +278,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int2 unit = tiles[(size_t)h * tmax + blockIdx.x];
   const int a = unit.x, r0 = unit.y;
   const int qend = q_off[(size_t)h * (Cq + 1) + a + 1];
+  const int nq = qend - r0 > BQ ? 2 : 1;  // query tiles of this block with rows
   const int ns = n_sel[(size_t)h * Cq + a];
   const int32_t* sl = sel + ((size_t)h * Cq + a) * Ck;
   const int32_t* koff = k_off + (size_t)h * (Ck + 1);
@@ -291,7 +290,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc::mbar_init(q_full, kProducers);
     for (int i = 0; i < kKSlots; ++i) {
       tc::mbar_init(k_full + i, 1);   // one arrival carrying the stage's byte count
-      tc::mbar_init(k_empty + i, 1);
+      tc::mbar_init(k_empty + i, 1 + 4 * nq);  // the MMA commit and one lane of each softmax warp
     }
     for (int i = 0; i < kVSlots; ++i) {
       tc::mbar_init(v_full + i, 1);
@@ -302,7 +301,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc::mbar_init(p_full + i, 128);
       tc::mbar_init(o_done + i, 1);
     }
-    tc::mbar_init(l_bar, 256);
     tc::mbar_init(done, 1);
     *abort_flag = 0;
     tc::mbar_fence_init();
@@ -370,38 +368,18 @@ __global__ void __launch_bounds__(kThreads, 1)
       // descriptors are built once; a K step only moves the start-address
       // field (address >> 4): +2 per 32 B inside a swizzled row, +1024 per
       // 16 KB region of Q, +16 per 256 B of a K tile, +2*kGroup/16 for V
-      const uint64_t qd = tc::desc_kmajor(tc::smem_u32(smem + S::q_off), BQ * 128u, 0);
+      const uint64_t qd0 = tc::desc_kmajor(tc::smem_u32(smem + S::q_off), BQ * 128u, 0);
       const uint64_t kd0 = tc::desc_kmajor_g8(tc::smem_u32(smem + S::k_off), kGroup, 0);
       const uint64_t vd0 = tc::desc_mnmajor_g8(tc::smem_u32(smem + S::v_off), kGroup, 0);
       constexpr uint64_t kStageStep = (uint64_t)(S::kKTile >> 4);
+      constexpr uint64_t kQStep = (uint64_t)(S::kQTile >> 4);
       bool ok = tc::mbar_wait(q_full, 0, abort_flag, status);
-      auto issue_pv = [&](int j) -> bool {
-        const int b = j & 1, u0 = ustart(j), np = nparts(j);
-        for (int p = 0; p < np; ++p)
-          if (!tc::mbar_wait(v_full + (u0 + p) % kVSlots, ((u0 + p) / kVSlots) & 1, abort_flag, status)) return false;
-        if (!tc::mbar_wait(p_full + b, (j >> 1) & 1, abort_flag, status)) return false;
-        tc::tc_fence_after();
-        const uint32_t pcol = tmem + kColS + (uint32_t)(b * 128);
-        const uint32_t ocol = tmem + kColO + (uint32_t)(b * D);  // O[b]: the stages of softmax group b
-        for (int p = 0; p < np; ++p) {
-          const uint64_t vd = vd0 + (uint64_t)((u0 + p) % kVSlots) * kStageStep;
-#pragma unroll
-          for (int k = 0; k < BN / 16; ++k)
-            tc::mma_ts(ocol, pcol + (uint32_t)k * 8u, vd + (uint64_t)k * (2u * kGroup >> 4), id_o,
-                       (j > 1 || p > 0 || k > 0) ? 1u : 0u);
-        }
-        tc::mma_commit(o_done + b);
-        for (int p = 0; p < np; ++p) tc::mma_commit(v_empty + (u0 + p) % kVSlots);
-        return true;
-      };
-      for (int j = 0; ok && j < ntile; ++j) {
-        const int b = j & 1, u0 = ustart(j), np = nparts(j);
-        for (int p = 0; ok && p < np; ++p)
-          ok = tc::mbar_wait(k_full + (u0 + p) % kKSlots, ((u0 + p) / kKSlots) & 1, abort_flag, status);
-        if (!ok) break;
-        tc::tc_fence_after();
-        // S[b] was last read as P[b] by P.V of tile j-2, issued before
-        const uint32_t scol = tmem + kColS + (uint32_t)(b * 128);
+      // S[t] = Q_t K_j^T (all parts of stage j); S[t] was last read as P[t]
+      // by P.V_t(j - 1), issued before
+      auto issue_s = [&](int t, int j) {
+        const int u0 = ustart(j), np = nparts(j);
+        const uint32_t scol = tmem + kColS + (uint32_t)(t * 128);
+        const uint64_t qd = qd0 + (uint64_t)t * kQStep;
         for (int p = 0; p < np; ++p) {
           const uint64_t kd = kd0 + (uint64_t)((u0 + p) % kKSlots) * kStageStep;
 #pragma unroll
@@ -409,11 +387,51 @@ __global__ void __launch_bounds__(kThreads, 1)
             tc::mma_ss(scol, qd + (uint64_t)((k >> 2) * 1024 + (k & 3) * 2), kd + (uint64_t)k * 16u, id_s,
                        (p > 0 || k > 0) ? 1u : 0u);
         }
-        tc::mma_commit(s_full + b);
-        for (int p = 0; p < np; ++p) tc::mma_commit(k_empty + (u0 + p) % kKSlots);
-        if (j > 0 && !issue_pv(j - 1)) { ok = false; break; }
+        tc::mma_commit(s_full + t);
+      };
+      auto wait_k = [&](int j) -> bool {
+        const int u0 = ustart(j), np = nparts(j);
+        for (int p = 0; p < np; ++p)
+          if (!tc::mbar_wait(k_full + (u0 + p) % kKSlots, ((u0 + p) / kKSlots) & 1, abort_flag, status)) return false;
+        tc::tc_fence_after();
+        return true;
+      };
+      if (ok && ntile > 0) {
+        ok = wait_k(0);
+        if (ok) {
+          for (int t = 0; t < nq; ++t) issue_s(t, 0);
+          for (int p = 0; p < nparts(0); ++p) tc::mma_commit(k_empty + (ustart(0) + p) % kKSlots);
+        }
       }
-      if (ok && ntile > 0) issue_pv(ntile - 1);
+      for (int j = 0; ok && j < ntile; ++j) {
+        const int u0 = ustart(j), np = nparts(j);
+        for (int p = 0; ok && p < np; ++p)
+          ok = tc::mbar_wait(v_full + (u0 + p) % kVSlots, ((u0 + p) / kVSlots) & 1, abort_flag, status);
+        for (int t = 0; ok && t < nq; ++t) {
+          // O[t] += P[t] V_j once the softmax of tile t has written P[t]
+          if (!tc::mbar_wait(p_full + t, j & 1, abort_flag, status)) { ok = false; break; }
+          tc::tc_fence_after();
+          const uint32_t pcol = tmem + kColS + (uint32_t)(t * 128);
+          const uint32_t ocol = tmem + kColO + (uint32_t)(t * D);
+          for (int p = 0; p < np; ++p) {
+            const uint64_t vd = vd0 + (uint64_t)((u0 + p) % kVSlots) * kStageStep;
+#pragma unroll
+            for (int k = 0; k < BN / 16; ++k)
+              tc::mma_ts(ocol, pcol + (uint32_t)k * 8u, vd + (uint64_t)k * (2u * kGroup >> 4), id_o,
+                         (j > 0 || p > 0 || k > 0) ? 1u : 0u);
+          }
+          tc::mma_commit(o_done + t);
+          if (t == nq - 1)
+            for (int p = 0; p < np; ++p) tc::mma_commit(v_empty + (u0 + p) % kVSlots);
+          // then S of the next stage for the same tile
+          if (j + 1 < ntile) {
+            if (t == 0 && !wait_k(j + 1)) { ok = false; break; }
+            issue_s(t, j + 1);
+            if (t == nq - 1)
+              for (int p = 0; p < nparts(j + 1); ++p) tc::mma_commit(k_empty + (ustart(j + 1) + p) % kKSlots);
+          }
+        }
+      }
       tc::mma_commit(done);
     }
     __syncwarp();
@@ -423,11 +441,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     {
       const bf16* Qh = Qp + (size_t)h * Nq * D;
       const uint32_t qa = tc::smem_u32(smem + S::q_off);
-      for (int e = pt; e < BQ * CPR; e += kProducers) {
+      // both query tiles (rows past the cluster's end are zero)
+      for (int e = pt; e < 2 * BQ * CPR; e += kProducers) {
         const int r = e / CPR, c = e % CPR, row = r0 + r;
         const bool valid = row < qend;
-        tc::cp_async16(qa + tc::sw128_offset(r, c, BQ), Qh + (size_t)(valid ? row : 0) * D + c * 8,
-                       valid ? 16u : 0u);
+        tc::cp_async16(qa + (uint32_t)(r / BQ) * (uint32_t)S::kQTile + tc::sw128_offset(r % BQ, c, BQ),
+                       Qh + (size_t)(valid ? row : 0) * D + c * 8, valid ? 16u : 0u);
       }
       tc::cp_async_wait_all();
       tc::fence_proxy_async();
@@ -504,10 +523,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       return npc;
     };
     // warp 1 produces the even stages, warp 2 the odd ones (warp 3 only helps
-    // with the query tile): keys once the K slot is free, then values, bias
-    // and mask once the V slot is.  A warp reaches stage u only after its
-    // stage u - 2 saw P.V of stage u - 4 complete, so every S and P.V up to
-    // there is done and no wait on a ring barrier can run a phase ahead.
+    // with the query tile): keys and the stage's bias once the K slot is free,
+    // then values once the V slot is.  A warp reaches stage u only after its
+    // stage u - 2 saw P.V of stage u - 4 complete, so every S, softmax and P.V
+    // up to there is done and no wait on a ring barrier can run a phase ahead.
     if (warp == 1 || warp == 2) {
       const int pw = warp - 1;
       int4* pcs = pieces + pw * kMaxPieces;  // this warp's piece list
@@ -530,10 +549,18 @@ __global__ void __launch_bounds__(kThreads, 1)
         uint8_t* vtile = smem + S::v_off + st * S::kKTile;
         int npc = 0, tail = BN;
         uint32_t bytes = 0;
-        // ---- keys
+        // ---- keys, bias and mask
         if (!tc::mbar_wait_warp(k_empty + sk, ((u / kKSlots) & 1) ^ 1, abort_flag, status)) break;
+        float* bias = bias_s + sk * BN;
         if (exact) {
           npc = make_pieces(j * BN, pcs, tail, bytes);
+          // bias: valid keys 0, padding and the stream tail -inf
+          for (int i = lane; i < BN; i += 32) bias[i] = -INFINITY;
+          __syncwarp();
+          for (int q = 0; q < npc; ++q) {
+            const int4 pc = pcs[q];
+            for (int i = lane; i < pc.w; i += 32) bias[pc.x * 8 + i] = 0.f;
+          }
           // zero the rows past the stream end so the MMAs see finite values
           if (tail < BN) {
             uint4* zr = reinterpret_cast<uint4*>(ktile) + (tail >> 3) * (kGroup / 16);
@@ -551,31 +578,34 @@ __global__ void __launch_bounds__(kThreads, 1)
                              (uint32_t)pc.z * kGroup, k_full + sk);
             }
           }
-        } else if (lane == 0) {
-          const uint32_t n = (uint32_t)(BN / 8) * kGroup;
-          const size_t go = cbase + (size_t)(((j - n_ex) * BN) >> 3) * kGroup;
-          tc::mbar_arrive_expect_tx(k_full + sk, n);
-          tc::bulk_g2s(tc::smem_u32(ktile), (p == 0 ? kb_hi : kb_lo) + go, n, k_full + sk);
+        } else {
+          // a compensation tile's bias rides with its first (hi) part
+          if (p == 0) {
+            const int c0 = (j - n_ex) * BN;
+            for (int i = lane; i < BN; i += 32) {
+              const int c = c0 + i;
+              const bool routed = c < Ck && ((bits[c >> 5] >> (c & 31)) & 1u);
+              bias[i] = routed ? -INFINITY : LC[c];
+            }
+          }
+          __syncwarp();
+          if (lane == 0) {
+            const uint32_t n = (uint32_t)(BN / 8) * kGroup;
+            const size_t go = cbase + (size_t)(((j - n_ex) * BN) >> 3) * kGroup;
+            tc::mbar_arrive_expect_tx(k_full + sk, n);
+            tc::bulk_g2s(tc::smem_u32(ktile), (p == 0 ? kb_hi : kb_lo) + go, n, k_full + sk);
+          }
         }
         __syncwarp();
-        // ---- values, bias and mask
+        // ---- values
         if (!tc::mbar_wait_warp(v_empty + st, ((u / kVSlots) & 1) ^ 1, abort_flag, status)) break;
-        float* bias = bias_s + st * BN;
         if (exact) {
-          // bias: valid keys 0, padding and the stream tail -inf
-          for (int i = lane; i < BN; i += 32) bias[i] = -INFINITY;
-          __syncwarp();
-          for (int q = 0; q < npc; ++q) {
-            const int4 pc = pcs[q];
-            for (int i = lane; i < pc.w; i += 32) bias[pc.x * 8 + i] = 0.f;
-          }
           if (tail < BN) {
             uint4* zr = reinterpret_cast<uint4*>(vtile) + (tail >> 3) * (kGroup / 16);
             const int nz = ((BN - tail) >> 3) * (int)(kGroup / 16);
             for (int i = lane; i < nz; i += 32) zr[i] = make_uint4(0, 0, 0, 0);
             tc::fence_proxy_async();
           }
-          if (lane == 0) flag_s[st] = 1;
           __syncwarp();
           if (lane == 0) {
             tc::mbar_arrive_expect_tx(v_full + st, bytes);
@@ -586,47 +616,35 @@ __global__ void __launch_bounds__(kThreads, 1)
                              (uint32_t)pc.z * kGroup, v_full + st);
             }
           }
-        } else {
-          const int c0 = (j - n_ex) * BN;
-          if (p == 0) {
-            for (int i = lane; i < BN; i += 32) {
-              const int c = c0 + i;
-              const bool routed = c < Ck && ((bits[c >> 5] >> (c & 31)) & 1u);
-              bias[i] = routed ? -INFINITY : LC[c];
-            }
-            if (lane == 0) flag_s[st] = 1;
-          }
-          __syncwarp();
-          if (lane == 0) {
-            const uint32_t n = (uint32_t)(BN / 8) * kGroup;
-            const size_t go = cbase + (size_t)(c0 >> 3) * kGroup;
-            tc::mbar_arrive_expect_tx(v_full + st, n);
-            tc::bulk_g2s(tc::smem_u32(vtile), (p == 0 ? vb_hi : vb_lo) + go, n, v_full + st);
-          }
+        } else if (lane == 0) {
+          const uint32_t n = (uint32_t)(BN / 8) * kGroup;
+          const size_t go = cbase + (size_t)(((j - n_ex) * BN) >> 3) * kGroup;
+          tc::mbar_arrive_expect_tx(v_full + st, n);
+          tc::bulk_g2s(tc::smem_u32(vtile), (p == 0 ? vb_hi : vb_lo) + go, n, v_full + st);
         }
         __syncwarp();
       }
     }
-  } else {
+  } else if (warp < 8 || nq == 2) {
     // -------------------------------------------------------------- softmax
-    // group w (warps 4-7: w = 0, warps 8-11: w = 1) takes the stages j with
-    // j % 2 == w: S[w], its own running maximum m_w, row sum l_w and
-    // accumulator O[w]; the two partial results are merged at the end.
-    const int w = (warp - 4) >> 2;
+    // group t (warps 4-7: t = 0, warps 8-11: t = 1) owns query tile t: S[t],
+    // its running maximum m, row sum l and accumulator O[t], over every stage.
+    const int t = (warp - 4) >> 2;
     const int r = ((warp & 3) << 5) + lane;   // tile row == TMEM lane
     const uint32_t lane_base = (uint32_t)((warp & 3) << 5) << 16;
-    const uint32_t scol = kColS + (uint32_t)(w * 128);
-    const uint32_t ocol = kColO + (uint32_t)(w * D);
+    const uint32_t scol = kColS + (uint32_t)(t * 128);
+    const uint32_t ocol = kColO + (uint32_t)(t * D);
     float m_used = -INFINITY, l = 0.f;
     bool ok = true;
-    for (int j = w; ok && j < ntile; j += 2) {
-      const int u0 = ustart(j), st = u0 % kVSlots;
-      if (!tc::mbar_wait_warp(s_full + w, (j >> 1) & 1, abort_flag, status)) { ok = false; break; }
-      // bias / mask of this stage: acquire the producers' writes through the
-      // stage's V barrier (its next phase needs this stage's P.V first)
-      if (!tc::mbar_wait_warp(v_full + st, (u0 / kVSlots) & 1, abort_flag, status)) { ok = false; break; }
+    for (int j = 0; ok && j < ntile; ++j) {
+      const int u0 = ustart(j), sk = u0 % kKSlots;
+      if (!tc::mbar_wait_warp(s_full + t, j & 1, abort_flag, status)) { ok = false; break; }
+      // bias / mask of this stage: acquire the producer's writes through the
+      // stage's K barrier (already complete, since S was computed from it; its
+      // next phase needs this warp's arrival on the slot's empty barrier)
+      if (!tc::mbar_wait_warp(k_full + sk, (u0 / kKSlots) & 1, abort_flag, status)) { ok = false; break; }
       tc::tc_fence_after();
-      const float* bias = bias_s + st * BN;
+      const float* bias = bias_s + sk * BN;
       // the stage's 128 logits of this row, read once: x = s*log2e * S + bias
       uint32_t v[128];
       tc::tmem_ld32(tmem + lane_base + scol, *reinterpret_cast<uint32_t(*)[32]>(v));
@@ -655,13 +673,18 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         mx = fmaxf(tc::fmax3(m8[0], m8[1], m8[2]), tc::fmax3(tc::fmax3(m8[3], m8[4], m8[5]), m8[6], m8[7]));
       }
-      // lazy rescale: a row whose maximum grew by more than 2^8 rescales O[w]
-      // and l_w.  The tensor-memory accesses are warp-collective, so the warp
-      // rescales together (factor 1 for rows that do not need it).
+      // the bias is read: release the stage's K slot(s) on this warp's behalf
+      __syncwarp();
+      if (lane == 0)
+        for (int q = 0; q < nparts(j); ++q) tc::mbar_arrive(k_empty + (u0 + q) % kKSlots);
+      // lazy rescale: a row whose maximum grew by more than 2^8 rescales O[t]
+      // and l.  The tensor-memory accesses are warp-collective, so the warp
+      // rescales together (factor 1 for rows that do not need it).  O[t] is
+      // complete up to P.V_t(j - 1): S[t] of this stage was issued after it.
       const bool grow = mx > m_used + 8.f;
-      const bool has_o = j >= 2 && m_used > -INFINITY;
+      const bool has_o = j >= 1 && m_used > -INFINITY;
       if (__any_sync(0xffffffffu, grow && has_o)) {
-        if (!tc::mbar_wait_warp(o_done + w, ((j >> 1) - 1) & 1, abort_flag, status)) { ok = false; break; }
+        if (!tc::mbar_wait_warp(o_done + t, (j - 1) & 1, abort_flag, status)) { ok = false; break; }
         tc::tc_fence_after();
         const float f = (grow && has_o) ? ex2(m_used - mx) : 1.f;
 #pragma unroll
@@ -697,54 +720,31 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc::tmem_st_wait();
       l += ((r8[0] + r8[1]) + (r8[2] + r8[3])) + ((r8[4] + r8[5]) + (r8[6] + r8[7]));
       tc::tc_fence_before();
-      tc::mbar_arrive(p_full + w);
+      tc::mbar_arrive(p_full + t);
     }
-    // epilogue: merge the two groups' (m, l, O), normalise, store via perm_q.
-    // Group w writes the columns [w d/2, w d/2 + d/2) of the output rows.
-    if (ok) {
-      mx_s[w * BQ + r] = m_used;
-      ls_s[w * BQ + r] = l;
-      tc::mbar_arrive(l_bar);
-      ok = tc::mbar_wait_warp(l_bar, 0, abort_flag, status);
-    }
-    // the last P.V into each accumulator
-    for (int x = 0; ok && x < 2; ++x) {
-      const int jl = ntile - 1 - ((ntile - 1 - x) & 1);  // last stage with j % 2 == x
-      if (jl >= 0) ok = tc::mbar_wait_warp(o_done + x, (jl >> 1) & 1, abort_flag, status);
-    }
+    // epilogue: the last P.V into O[t], then O / l stored via perm_q
+    if (ok && ntile > 0) ok = tc::mbar_wait_warp(o_done + t, (ntile - 1) & 1, abort_flag, status);
     if (ok) {
       tc::tc_fence_after();
-      const float m0 = mx_s[r], m1 = mx_s[BQ + r];
-      const float mm = fmaxf(m0, m1);
-      // a group that saw no key (or no stage) contributes nothing; its
-      // accumulator is not read
-      const bool u0ok = m0 > -INFINITY, u1ok = m1 > -INFINITY;
-      const float a0 = u0ok ? ex2(m0 - mm) : 0.f, a1 = u1ok ? ex2(m1 - mm) : 0.f;
-      const float lt = ls_s[r] * a0 + ls_s[BQ + r] * a1;
-      const float inv = lt > 0.f ? 1.f / lt : 0.f;
-      const float f0 = a0 * inv, f1 = a1 * inv;
-      const int row = r0 + r;
+      // a row that saw no key (every logit masked) stores zeros
+      const bool have = m_used > -INFINITY && l > 0.f;
+      const float inv = have ? 1.f / l : 0.f;
+      const int row = r0 + t * BQ + r;
       const bool valid = row < qend;
-      constexpr int OH = D / 2;
-      bf16* orow = O + ((size_t)h * Nq + (valid ? perm_q[(size_t)h * Nq + row] : 0)) * D + w * OH;
+      bf16* orow = O + ((size_t)h * Nq + (valid ? perm_q[(size_t)h * Nq + row] : 0)) * D;
 #pragma unroll
-      for (int q = 0; q < OH / 16; ++q) {
-        uint32_t o0[16], o1[16];
-        tc::tmem_ld16(tmem + lane_base + kColO + (uint32_t)(w * OH + q * 16), o0);
-        tc::tmem_ld16(tmem + lane_base + kColO + (uint32_t)(D + w * OH + q * 16), o1);
+      for (int q = 0; q < D / 32; ++q) {
+        uint32_t o[32];
+        tc::tmem_ld32(tmem + lane_base + ocol + (uint32_t)(q * 32), o);
         tc::tmem_ld_wait();
-        float o[16];
+        uint4 w4[4];
+        uint32_t* wp = reinterpret_cast<uint32_t*>(w4);
 #pragma unroll
         for (int i = 0; i < 16; ++i)
-          o[i] = (u0ok ? __uint_as_float(o0[i]) * f0 : 0.f) + (u1ok ? __uint_as_float(o1[i]) * f1 : 0.f);
-        uint4 w0, w1;
-        w0.x = pack_bf16(o[0], o[1]); w0.y = pack_bf16(o[2], o[3]);
-        w0.z = pack_bf16(o[4], o[5]); w0.w = pack_bf16(o[6], o[7]);
-        w1.x = pack_bf16(o[8], o[9]); w1.y = pack_bf16(o[10], o[11]);
-        w1.z = pack_bf16(o[12], o[13]); w1.w = pack_bf16(o[14], o[15]);
+          wp[i] = have ? pack_bf16(__uint_as_float(o[2 * i]) * inv, __uint_as_float(o[2 * i + 1]) * inv) : 0u;
         if (valid) {
-          reinterpret_cast<uint4*>(orow + q * 16)[0] = w0;
-          reinterpret_cast<uint4*>(orow + q * 16)[1] = w1;
+#pragma unroll
+          for (int i = 0; i < 4; ++i) reinterpret_cast<uint4*>(orow + q * 32)[i] = w4[i];
         }
       }
     }
