@@ -20,12 +20,13 @@
 // padded to a multiple of 8 rows, each group of 8 rows stored as
 // [16-byte chunk][row]), which is directly a no-swizzle UMMA operand (K-major
 // for K, MN-major for V); a stage is one or a few contiguous runs, each moved
-// by a single cp.async.bulk.  K (with the stage's bias vector) and V each have
-// a two-slot ring: a K slot is free once S of its stage is computed for both
-// query tiles and both softmax groups have read the bias, a V slot once P.V is
-// done for both tiles; padding rows are masked through the bias.  A softmax
-// stage waits only for its S (and the bias that came with the keys), never for
-// the values, which load while it runs.  Sharing each stage between two query
+// by a single cp.async.bulk.  K and V each have a two-slot ring: a K slot is
+// free once S of its stage is computed for both query tiles, a V slot once
+// P.V is done for both tiles.  The stage's bias vector (padding rows and
+// routed centroids masked, log2|k_c| on compensated centroids) has a
+// four-slot ring of its own, freed by the softmax warps once they have read
+// it, so keys for later stages load while the softmax of this one runs, and a
+// softmax stage never waits for the values.  Sharing each stage between two query
 // tiles halves the key / value traffic from L2 per FLOP, which is what bounds
 // a one-tile block.
 // Warp roles (12 warps):
@@ -60,7 +61,8 @@ constexpr int BQ = 128;        // rows per query tile (two tiles per block)
 constexpr int BN = 128;        // keys per ring stage
 constexpr int kThreads = 384;
 constexpr int kProducers = 96;
-constexpr int kKSlots = 2;     // K ring, with the stage's bias vector
+constexpr int kKSlots = 2;     // K ring
+constexpr int kBSlots = 4;     // bias ring
 constexpr int kVSlots = 2;     // V ring
 constexpr int kUnitRows = 2 * BQ;  // query rows of one block
 constexpr float kLog2e = 1.4426950408889634f;
@@ -227,8 +229,8 @@ struct AttnSmem {
   static constexpr int q_off = 0;                                    // [2] query tiles
   static constexpr int k_off = q_off + 2 * kQTile;                   // [kKSlots] key tiles
   static constexpr int v_off = k_off + kKSlots * kKTile;             // [kVSlots] value tiles
-  static constexpr int bias_off = v_off + kVSlots * kKTile;          // [kKSlots][BN] log2 biases
-  static constexpr int bits_off = bias_off + kKSlots * BN * 4;
+  static constexpr int bias_off = v_off + kVSlots * kKTile;          // [kBSlots][BN] log2 biases
+  static constexpr int bits_off = bias_off + kBSlots * BN * 4;
   static constexpr int rng_off = bits_off + kMaxCkBits / 8;          // [3][kMaxRanges] start, prefix, len
   static constexpr int pc_off = rng_off + 3 * kMaxRanges * 4 + 16;   // [producer warp][32] piece lists
   static constexpr int bar_off = pc_off + 2 * 32 * 16;
@@ -265,15 +267,17 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + S::bar_off);
   uint64_t* q_full = bars + 0;
   uint64_t* k_full = bars + 1;     // [kKSlots]
-  uint64_t* k_empty = bars + 4;    // [kKSlots]: S of the stage done + its bias read by every softmax warp
+  uint64_t* k_empty = bars + 4;    // [kKSlots]
   uint64_t* v_full = bars + 7;     // [kVSlots]
   uint64_t* v_empty = bars + 9;    // [kVSlots]
   uint64_t* s_full = bars + 11;    // [2 query tiles]
   uint64_t* p_full = bars + 13;    // [2 query tiles]
   uint64_t* o_done = bars + 15;    // [2 query tiles]
   uint64_t* done = bars + 18;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 19);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 20);
+  uint64_t* b_full = bars + 19;    // [kBSlots]
+  uint64_t* b_empty = bars + 23;   // [kBSlots]: read by one lane of every softmax warp
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 27);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 28);
 
   const int2 unit = tiles[(size_t)h * tmax + blockIdx.x];
   const int a = unit.x, r0 = unit.y;
@@ -290,7 +294,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc::mbar_init(q_full, kProducers);
     for (int i = 0; i < kKSlots; ++i) {
       tc::mbar_init(k_full + i, 1);   // one arrival carrying the stage's byte count
-      tc::mbar_init(k_empty + i, 1 + 4 * nq);  // the MMA commit and one lane of each softmax warp
+      tc::mbar_init(k_empty + i, 1);
     }
     for (int i = 0; i < kVSlots; ++i) {
       tc::mbar_init(v_full + i, 1);
@@ -302,6 +306,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc::mbar_init(o_done + i, 1);
     }
     tc::mbar_init(done, 1);
+    for (int i = 0; i < kBSlots; ++i) {
+      tc::mbar_init(b_full + i, 1);
+      tc::mbar_init(b_empty + i, 4 * nq);
+    }
     *abort_flag = 0;
     tc::mbar_fence_init();
   }
@@ -362,78 +370,90 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (warp == 0) {
     // ------------------------------------------------------------------ MMA
-    if (lane == 0) {
-      const uint32_t id_s = tc::idesc_bf16(BQ, BN, false, false);
-      const uint32_t id_o = tc::idesc_bf16(BQ, D, false, true);
-      // descriptors are built once; a K step only moves the start-address
-      // field (address >> 4): +2 per 32 B inside a swizzled row, +1024 per
-      // 16 KB region of Q, +16 per 256 B of a K tile, +2*kGroup/16 for V
-      const uint64_t qd0 = tc::desc_kmajor(tc::smem_u32(smem + S::q_off), BQ * 128u, 0);
-      const uint64_t kd0 = tc::desc_kmajor_g8(tc::smem_u32(smem + S::k_off), kGroup, 0);
-      const uint64_t vd0 = tc::desc_mnmajor_g8(tc::smem_u32(smem + S::v_off), kGroup, 0);
-      constexpr uint64_t kStageStep = (uint64_t)(S::kKTile >> 4);
-      constexpr uint64_t kQStep = (uint64_t)(S::kQTile >> 4);
-      bool ok = tc::mbar_wait(q_full, 0, abort_flag, status);
-      // S[t] = Q_t K_j^T (all parts of stage j); S[t] was last read as P[t]
-      // by P.V_t(j - 1), issued before
-      auto issue_s = [&](int t, int j) {
-        const int u0 = ustart(j), np = nparts(j);
-        const uint32_t scol = tmem + kColS + (uint32_t)(t * 128);
-        const uint64_t qd = qd0 + (uint64_t)t * kQStep;
-        for (int p = 0; p < np; ++p) {
-          const uint64_t kd = kd0 + (uint64_t)((u0 + p) % kKSlots) * kStageStep;
+    // The whole warp runs the issue loop, so the loop control and the
+    // descriptor arithmetic are warp-uniform; one elected lane issues each
+    // tcgen05.mma and commit.  Every wait is made warp-uniform.
+    const bool leader = tc::elect_one();
+    const uint32_t id_s = tc::idesc_bf16(BQ, BN, false, false);
+    const uint32_t id_o = tc::idesc_bf16(BQ, D, false, true);
+    // descriptors are built once; a K step only moves the start-address
+    // field (address >> 4): +2 per 32 B inside a swizzled row, +1024 per
+    // 16 KB region of Q, +16 per 256 B of a K tile, +2*kGroup/16 for V
+    const uint64_t qd0 = tc::desc_kmajor(tc::smem_u32(smem + S::q_off), BQ * 128u, 0);
+    const uint64_t kd0 = tc::desc_kmajor_g8(tc::smem_u32(smem + S::k_off), kGroup, 0);
+    const uint64_t vd0 = tc::desc_mnmajor_g8(tc::smem_u32(smem + S::v_off), kGroup, 0);
+    constexpr uint64_t kStageStep = (uint64_t)(S::kKTile >> 4);
+    constexpr uint64_t kQStep = (uint64_t)(S::kQTile >> 4);
+    bool ok = tc::mbar_wait_warp(q_full, 0, abort_flag, status);
+    // S[t] = Q_t K_j^T (all parts of stage j); S[t] was last read as P[t]
+    // by P.V_t(j - 1), issued before
+    auto issue_s = [&](int t, int j) {
+      const int u0 = ustart(j), np = nparts(j);
+      const uint32_t scol = tmem + kColS + (uint32_t)(t * 128);
+      const uint64_t qd = qd0 + (uint64_t)t * kQStep;
+      for (int p = 0; p < np; ++p) {
+        const uint64_t kd = kd0 + (uint64_t)((u0 + p) % kKSlots) * kStageStep;
+        if (leader) {
 #pragma unroll
           for (int k = 0; k < D / 16; ++k)
             tc::mma_ss(scol, qd + (uint64_t)((k >> 2) * 1024 + (k & 3) * 2), kd + (uint64_t)k * 16u, id_s,
                        (p > 0 || k > 0) ? 1u : 0u);
         }
-        tc::mma_commit(s_full + t);
-      };
-      auto wait_k = [&](int j) -> bool {
-        const int u0 = ustart(j), np = nparts(j);
-        for (int p = 0; p < np; ++p)
-          if (!tc::mbar_wait(k_full + (u0 + p) % kKSlots, ((u0 + p) / kKSlots) & 1, abort_flag, status)) return false;
-        tc::tc_fence_after();
-        return true;
-      };
-      if (ok && ntile > 0) {
-        ok = wait_k(0);
-        if (ok) {
-          for (int t = 0; t < nq; ++t) issue_s(t, 0);
-          for (int p = 0; p < nparts(0); ++p) tc::mma_commit(k_empty + (ustart(0) + p) % kKSlots);
-        }
       }
-      for (int j = 0; ok && j < ntile; ++j) {
-        const int u0 = ustart(j), np = nparts(j);
-        for (int p = 0; ok && p < np; ++p)
-          ok = tc::mbar_wait(v_full + (u0 + p) % kVSlots, ((u0 + p) / kVSlots) & 1, abort_flag, status);
-        for (int t = 0; ok && t < nq; ++t) {
-          // O[t] += P[t] V_j once the softmax of tile t has written P[t]
-          if (!tc::mbar_wait(p_full + t, j & 1, abort_flag, status)) { ok = false; break; }
-          tc::tc_fence_after();
-          const uint32_t pcol = tmem + kColS + (uint32_t)(t * 128);
-          const uint32_t ocol = tmem + kColO + (uint32_t)(t * D);
-          for (int p = 0; p < np; ++p) {
-            const uint64_t vd = vd0 + (uint64_t)((u0 + p) % kVSlots) * kStageStep;
+      if (leader) tc::mma_commit(s_full + t);
+      __syncwarp();
+    };
+    auto wait_k = [&](int j) -> bool {
+      const int u0 = ustart(j), np = nparts(j);
+      for (int p = 0; p < np; ++p)
+        if (!tc::mbar_wait_warp(k_full + (u0 + p) % kKSlots, ((u0 + p) / kKSlots) & 1, abort_flag, status))
+          return false;
+      tc::tc_fence_after();
+      return true;
+    };
+    auto commit_slots = [&](uint64_t* ring, int nslots, int j) {
+      if (leader)
+        for (int p = 0; p < nparts(j); ++p) tc::mma_commit(ring + (ustart(j) + p) % nslots);
+      __syncwarp();
+    };
+    if (ok && ntile > 0) {
+      ok = wait_k(0);
+      if (ok) {
+        for (int t = 0; t < nq; ++t) issue_s(t, 0);
+        commit_slots(k_empty, kKSlots, 0);
+      }
+    }
+    for (int j = 0; ok && j < ntile; ++j) {
+      const int u0 = ustart(j), np = nparts(j);
+      for (int p = 0; ok && p < np; ++p)
+        ok = tc::mbar_wait_warp(v_full + (u0 + p) % kVSlots, ((u0 + p) / kVSlots) & 1, abort_flag, status);
+      for (int t = 0; ok && t < nq; ++t) {
+        // O[t] += P[t] V_j once the softmax of tile t has written P[t]
+        if (!tc::mbar_wait_warp(p_full + t, j & 1, abort_flag, status)) { ok = false; break; }
+        tc::tc_fence_after();
+        const uint32_t pcol = tmem + kColS + (uint32_t)(t * 128);
+        const uint32_t ocol = tmem + kColO + (uint32_t)(t * D);
+        for (int p = 0; p < np; ++p) {
+          const uint64_t vd = vd0 + (uint64_t)((u0 + p) % kVSlots) * kStageStep;
+          if (leader) {
 #pragma unroll
             for (int k = 0; k < BN / 16; ++k)
               tc::mma_ts(ocol, pcol + (uint32_t)k * 8u, vd + (uint64_t)k * (2u * kGroup >> 4), id_o,
                          (j > 0 || p > 0 || k > 0) ? 1u : 0u);
           }
-          tc::mma_commit(o_done + t);
-          if (t == nq - 1)
-            for (int p = 0; p < np; ++p) tc::mma_commit(v_empty + (u0 + p) % kVSlots);
-          // then S of the next stage for the same tile
-          if (j + 1 < ntile) {
-            if (t == 0 && !wait_k(j + 1)) { ok = false; break; }
-            issue_s(t, j + 1);
-            if (t == nq - 1)
-              for (int p = 0; p < nparts(j + 1); ++p) tc::mma_commit(k_empty + (ustart(j + 1) + p) % kKSlots);
-          }
+        }
+        if (leader) tc::mma_commit(o_done + t);
+        __syncwarp();
+        if (t == nq - 1) commit_slots(v_empty, kVSlots, j);
+        // then S of the next stage for the same tile
+        if (j + 1 < ntile) {
+          if (t == 0 && !wait_k(j + 1)) { ok = false; break; }
+          issue_s(t, j + 1);
+          if (t == nq - 1) commit_slots(k_empty, kKSlots, j + 1);
         }
       }
-      tc::mma_commit(done);
     }
+    if (leader) tc::mma_commit(done);
     __syncwarp();
   } else if (warp < 4) {
     // ------------------------------------------------------------ producers
@@ -523,10 +543,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       return npc;
     };
     // warp 1 produces the even stages, warp 2 the odd ones (warp 3 only helps
-    // with the query tile): keys and the stage's bias once the K slot is free,
-    // then values once the V slot is.  A warp reaches stage u only after its
-    // stage u - 2 saw P.V of stage u - 4 complete, so every S, softmax and P.V
-    // up to there is done and no wait on a ring barrier can run a phase ahead.
+    // with the query tile): keys once the K slot is free, the stage's bias
+    // once its bias slot is, then values once the V slot is.  Each warp always
+    // fills the same K and V slot and its own two bias slots, and it waits on
+    // a slot only for the stage it filled there last, so no wait on a ring
+    // barrier can run a phase ahead.
     if (warp == 1 || warp == 2) {
       const int pw = warp - 1;
       int4* pcs = pieces + pw * kMaxPieces;  // this warp's piece list
@@ -549,18 +570,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         uint8_t* vtile = smem + S::v_off + st * S::kKTile;
         int npc = 0, tail = BN;
         uint32_t bytes = 0;
-        // ---- keys, bias and mask
+        // ---- keys
         if (!tc::mbar_wait_warp(k_empty + sk, ((u / kKSlots) & 1) ^ 1, abort_flag, status)) break;
-        float* bias = bias_s + sk * BN;
         if (exact) {
           npc = make_pieces(j * BN, pcs, tail, bytes);
-          // bias: valid keys 0, padding and the stream tail -inf
-          for (int i = lane; i < BN; i += 32) bias[i] = -INFINITY;
-          __syncwarp();
-          for (int q = 0; q < npc; ++q) {
-            const int4 pc = pcs[q];
-            for (int i = lane; i < pc.w; i += 32) bias[pc.x * 8 + i] = 0.f;
-          }
           // zero the rows past the stream end so the MMAs see finite values
           if (tail < BN) {
             uint4* zr = reinterpret_cast<uint4*>(ktile) + (tail >> 3) * (kGroup / 16);
@@ -578,25 +591,36 @@ __global__ void __launch_bounds__(kThreads, 1)
                              (uint32_t)pc.z * kGroup, k_full + sk);
             }
           }
-        } else {
-          // a compensation tile's bias rides with its first (hi) part
-          if (p == 0) {
-            const int c0 = (j - n_ex) * BN;
-            for (int i = lane; i < BN; i += 32) {
-              const int c = c0 + i;
-              const bool routed = c < Ck && ((bits[c >> 5] >> (c & 31)) & 1u);
-              bias[i] = routed ? -INFINITY : LC[c];
-            }
-          }
+        } else if (lane == 0) {
+          const uint32_t n = (uint32_t)(BN / 8) * kGroup;
+          const size_t go = cbase + (size_t)(((j - n_ex) * BN) >> 3) * kGroup;
+          tc::mbar_arrive_expect_tx(k_full + sk, n);
+          tc::bulk_g2s(tc::smem_u32(ktile), (p == 0 ? kb_hi : kb_lo) + go, n, k_full + sk);
+        }
+        __syncwarp();
+        // ---- bias and mask (every ring stage passes through the bias ring;
+        // a compensation tile's bias rides with its first, hi, part)
+        const int sb = u % kBSlots;
+        if (!tc::mbar_wait_warp(b_empty + sb, ((u / kBSlots) & 1) ^ 1, abort_flag, status)) break;
+        float* bias = bias_s + sb * BN;
+        if (exact) {
+          // valid keys 0, padding and the stream tail -inf
+          for (int i = lane; i < BN; i += 32) bias[i] = -INFINITY;
           __syncwarp();
-          if (lane == 0) {
-            const uint32_t n = (uint32_t)(BN / 8) * kGroup;
-            const size_t go = cbase + (size_t)(((j - n_ex) * BN) >> 3) * kGroup;
-            tc::mbar_arrive_expect_tx(k_full + sk, n);
-            tc::bulk_g2s(tc::smem_u32(ktile), (p == 0 ? kb_hi : kb_lo) + go, n, k_full + sk);
+          for (int q = 0; q < npc; ++q) {
+            const int4 pc = pcs[q];
+            for (int i = lane; i < pc.w; i += 32) bias[pc.x * 8 + i] = 0.f;
+          }
+        } else if (p == 0) {
+          const int c0 = (j - n_ex) * BN;
+          for (int i = lane; i < BN; i += 32) {
+            const int c = c0 + i;
+            const bool routed = c < Ck && ((bits[c >> 5] >> (c & 31)) & 1u);
+            bias[i] = routed ? -INFINITY : LC[c];
           }
         }
         __syncwarp();
+        if (lane == 0) tc::mbar_arrive(b_full + sb);
         // ---- values
         if (!tc::mbar_wait_warp(v_empty + st, ((u / kVSlots) & 1) ^ 1, abort_flag, status)) break;
         if (exact) {
@@ -637,14 +661,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     float m_used = -INFINITY, l = 0.f;
     bool ok = true;
     for (int j = 0; ok && j < ntile; ++j) {
-      const int u0 = ustart(j), sk = u0 % kKSlots;
+      const int u0 = ustart(j), sb = u0 % kBSlots;
       if (!tc::mbar_wait_warp(s_full + t, j & 1, abort_flag, status)) { ok = false; break; }
-      // bias / mask of this stage: acquire the producer's writes through the
-      // stage's K barrier (already complete, since S was computed from it; its
-      // next phase needs this warp's arrival on the slot's empty barrier)
-      if (!tc::mbar_wait_warp(k_full + sk, (u0 / kKSlots) & 1, abort_flag, status)) { ok = false; break; }
+      // bias / mask of this stage (its next phase needs this warp's arrival
+      // on the slot's empty barrier, so the parity cannot run ahead)
+      if (!tc::mbar_wait_warp(b_full + sb, (u0 / kBSlots) & 1, abort_flag, status)) { ok = false; break; }
       tc::tc_fence_after();
-      const float* bias = bias_s + sk * BN;
+      const float* bias = bias_s + sb * BN;
       // the stage's 128 logits of this row, read once: x = s*log2e * S + bias
       uint32_t v[128];
       tc::tmem_ld32(tmem + lane_base + scol, *reinterpret_cast<uint32_t(*)[32]>(v));
@@ -673,10 +696,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         mx = fmaxf(tc::fmax3(m8[0], m8[1], m8[2]), tc::fmax3(tc::fmax3(m8[3], m8[4], m8[5]), m8[6], m8[7]));
       }
-      // the bias is read: release the stage's K slot(s) on this warp's behalf
+      // the bias is read: release the stage's bias slot(s) on this warp's behalf
       __syncwarp();
       if (lane == 0)
-        for (int q = 0; q < nparts(j); ++q) tc::mbar_arrive(k_empty + (u0 + q) % kKSlots);
+        for (int q = 0; q < nparts(j); ++q) tc::mbar_arrive(b_empty + (u0 + q) % kBSlots);
       // lazy rescale: a row whose maximum grew by more than 2^8 rescales O[t]
       // and l.  The tensor-memory accesses are warp-collective, so the warp
       // rescales together (factor 1 for rows that do not need it).  O[t] is

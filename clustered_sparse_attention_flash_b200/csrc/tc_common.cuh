@@ -93,6 +93,15 @@ __device__ __forceinline__ bool mbar_wait_warp(uint64_t* bar, uint32_t parity, v
   return __all_sync(0xffffffffu, ok);
 }
 
+// True on exactly one active lane of the warp (warp-collective).
+__device__ __forceinline__ bool elect_one() {
+  uint32_t p;
+  asm volatile(
+      "{\n\t.reg .pred P;\n\telect.sync _|P, 0xffffffff;\n\tselp.u32 %0, 1, 0, P;\n\t}"
+      : "=r"(p));
+  return p != 0;
+}
+
 // Named barrier `id` over `count` threads that also ANDs a predicate, so all
 // participants take the same branch afterwards.
 __device__ __forceinline__ bool bar_and(int id, int count, bool v) {
