@@ -149,31 +149,37 @@ __global__ void __launch_bounds__(kBeThreads, 1)
 
   if (warp == 0) {
     // ---------------------------------------------------------- MMA issuer
-    if (lane == 0 && ntiles > 0) {
-      bool ok = tc::mbar_wait(q_full, 0, abort_flag, status);
+    // The whole warp runs the loop (warp-uniform control and descriptor
+    // arithmetic); one elected lane issues each tcgen05.mma and commit.
+    const bool leader = tc::elect_one();
+    if (ntiles > 0) {
+      bool ok = tc::mbar_wait_warp(q_full, 0, abort_flag, status);
       const uint32_t qa = tc::smem_u32(q_s);
       const uint32_t id = tc::idesc_bf16(kBeRows, kBeKeys, false, false);
       for (int t = 0; ok && t < ntiles; ++t) {
         const int s = t % kBeStages, buf = t & 1;
-        ok = tc::mbar_wait(full + s, (t / kBeStages) & 1, abort_flag, status);
-        if (ok) ok = tc::mbar_wait(acc_empty + buf, ((t >> 1) & 1) ^ 1, abort_flag, status);
+        ok = tc::mbar_wait_warp(full + s, (t / kBeStages) & 1, abort_flag, status);
+        if (ok) ok = tc::mbar_wait_warp(acc_empty + buf, ((t >> 1) & 1) ^ 1, abort_flag, status);
         if (!ok) break;
         tc::tc_fence_after();
         const uint32_t ka = tc::smem_u32(k_s + s * kKStage);
         const uint32_t d_t = tmem + (uint32_t)(buf * kBeKeys);
+        if (leader) {
 #pragma unroll
-        for (int part = 0; part < 2; ++part)
+          for (int part = 0; part < 2; ++part)
 #pragma unroll
-          for (int k16 = 0; k16 < D / 16; ++k16) {
-            const uint64_t a = tc::desc_kmajor(qa + (uint32_t)(part * kQPart), kBeRows * 128u, k16);
-            const uint64_t b = tc::desc_kmajor(ka, kBeKeys * 128u, k16);
-            tc::mma_ss(d_t, a, b, id, (part | k16) ? 1u : 0u);
-          }
-        tc::mma_commit(acc_full + buf);
-        tc::mma_commit(empty + s);
+            for (int k16 = 0; k16 < D / 16; ++k16) {
+              const uint64_t a = tc::desc_kmajor(qa + (uint32_t)(part * kQPart), kBeRows * 128u, k16);
+              const uint64_t b = tc::desc_kmajor(ka, kBeKeys * 128u, k16);
+              tc::mma_ss(d_t, a, b, id, (part | k16) ? 1u : 0u);
+            }
+          tc::mma_commit(acc_full + buf);
+          tc::mma_commit(empty + s);
+        }
+        __syncwarp();
       }
     }
-    if (lane == 0) tc::mma_commit(done);
+    if (leader) tc::mma_commit(done);
     __syncwarp();
   } else if (warp == 1) {
     // ------------------------------------------- TMA copies and key scalars

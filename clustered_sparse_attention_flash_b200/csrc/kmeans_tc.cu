@@ -471,24 +471,27 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (warp == 0) {
     // ---------------------------------------------------------- MMA issuer
-    if (lane == 0) {
-      bool ok = tc::mbar_wait(cent_full, 0, abort_flag, status);
-      const uint32_t cent_a = tc::smem_u32(cent_s);
-      const uint32_t cregion = (uint32_t)Cr * 128u;
-      int g = 0;
-      for (int t = 0; ok && t < nt; ++t) {
-        const int s = t % stages, k = t / stages;
-        ok = tc::mbar_wait(x_full + s, k & 1, abort_flag, status);
+    // The whole warp runs the loop (warp-uniform control and descriptor
+    // arithmetic); one elected lane issues each tcgen05.mma and commit.
+    const bool leader = tc::elect_one();
+    bool ok = tc::mbar_wait_warp(cent_full, 0, abort_flag, status);
+    const uint32_t cent_a = tc::smem_u32(cent_s);
+    const uint32_t cregion = (uint32_t)Cr * 128u;
+    int g = 0;
+    for (int t = 0; ok && t < nt; ++t) {
+      const int s = t % stages, k = t / stages;
+      ok = tc::mbar_wait_warp(x_full + s, k & 1, abort_flag, status);
+      if (!ok) break;
+      tc::tc_fence_after();
+      const uint32_t xa = tc::smem_u32(x_s + s * kXBytes);
+      for (int j = 0; j < nch; ++j, ++g) {
+        const int slot = g & (kSlots - 1), use = g >> 2;
+        ok = tc::mbar_wait_warp(acc_empty + slot, (use & 1) ^ 1, abort_flag, status);
         if (!ok) break;
         tc::tc_fence_after();
-        const uint32_t xa = tc::smem_u32(x_s + s * kXBytes);
-        for (int j = 0; j < nch; ++j, ++g) {
-          const int slot = g & (kSlots - 1), use = g >> 2;
-          ok = tc::mbar_wait(acc_empty + slot, (use & 1) ^ 1, abort_flag, status);
-          if (!ok) break;
-          tc::tc_fence_after();
-          const int n0 = j * kChunk, nj = min(kChunk, Cpad - n0);
-          const uint32_t id = tc::idesc_bf16(BM, nj, false, false);
+        const int n0 = j * kChunk, nj = min(kChunk, Cpad - n0);
+        const uint32_t id = tc::idesc_bf16(BM, nj, false, false);
+        if (leader) {
 #pragma unroll
           for (int k16 = 0; k16 < D / 16; ++k16) {
             const uint64_t a = tc::desc_kmajor(xa, BM * 128u, k16);
@@ -497,11 +500,13 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           tc::mma_commit(acc_full + slot);
         }
-        if (!ok) break;
-        tc::mma_commit(x_empty + s);
+        __syncwarp();
       }
-      tc::mma_commit(done);
+      if (!ok) break;
+      if (leader) tc::mma_commit(x_empty + s);
+      __syncwarp();
     }
+    if (leader) tc::mma_commit(done);
     __syncwarp();
   } else if (warp == 1) {
     // --------------------------------------------------------- TMA producer
