@@ -79,6 +79,34 @@ __device__ __forceinline__ float ex2(float x) {
   return y;
 }
 
+// Packed pairs of float32 (sm_100 two-wide FMA pipe): one instruction
+// applies the same operation to both halves, rounded as the scalar one.
+__device__ __forceinline__ uint64_t f2(float lo, float hi) {
+  uint64_t d;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(d) : "f"(lo), "f"(hi));
+  return d;
+}
+__device__ __forceinline__ float f2_lo(uint64_t x) {
+  float lo, hi;
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(x));
+  return lo;
+}
+__device__ __forceinline__ float f2_hi(uint64_t x) {
+  float lo, hi;
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(x));
+  return hi;
+}
+__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+__device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   uint32_t r;
   asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
@@ -677,6 +705,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc::tmem_ld_wait();
       float mx;
       {
+        const uint64_t sc2 = f2(scale2, scale2);
         float m8[8];
 #pragma unroll
         for (int k = 0; k < 8; ++k) m8[k] = -INFINITY;
@@ -689,10 +718,14 @@ __global__ void __launch_bounds__(kThreads, 1)
           const float bb[16] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w,
                                 b2.x, b2.y, b2.z, b2.w, b3.x, b3.y, b3.z, b3.w};
 #pragma unroll
-          for (int k = 0; k < 16; ++k) v[i + k] = __float_as_uint(fmaf(__uint_as_float(v[i + k]), scale2, bb[k]));
-#pragma unroll
-          for (int k = 0; k < 8; ++k)
-            m8[k] = tc::fmax3(m8[k], __uint_as_float(v[i + k]), __uint_as_float(v[i + 8 + k]));
+          for (int k = 0; k < 8; ++k) {
+            // x = s * scale2 + bias for two keys per instruction
+            const uint64_t x = f2_fma(f2(__uint_as_float(v[i + 2 * k]), __uint_as_float(v[i + 2 * k + 1])), sc2,
+                                      f2(bb[2 * k], bb[2 * k + 1]));
+            v[i + 2 * k] = __float_as_uint(f2_lo(x));
+            v[i + 2 * k + 1] = __float_as_uint(f2_hi(x));
+            m8[k] = tc::fmax3(m8[k], f2_lo(x), f2_hi(x));
+          }
         }
         mx = fmaxf(tc::fmax3(m8[0], m8[1], m8[2]), tc::fmax3(tc::fmax3(m8[3], m8[4], m8[5]), m8[6], m8[7]));
       }
@@ -724,24 +757,29 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       if (grow) m_used = mx;
       const float mref = m_used == -INFINITY ? 0.f : m_used;
-      // P = 2^(x - m) in bf16 over the first 64 columns of S[w] (keys 2c and
+      // P = 2^(x - m) in bf16 over the first 64 columns of S[t] (keys 2c and
       // 2c + 1 in column c; every S value of the row is already in registers)
-      float r8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+      // (x - m for two keys per instruction; row sums in four packed pairs)
+      const uint64_t negm = f2(-mref, -mref);
+      uint64_t r4[4] = {0ull, 0ull, 0ull, 0ull};
 #pragma unroll
       for (int q = 0; q < 4; ++q) {
         uint32_t pk[16];
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
           const int c = q * 32 + 2 * i;
-          const float p0 = ex2(__uint_as_float(v[c]) - mref);
-          const float p1 = ex2(__uint_as_float(v[c + 1]) - mref);
-          r8[i & 7] += p0 + p1;
+          const uint64_t x = f2_add(f2(__uint_as_float(v[c]), __uint_as_float(v[c + 1])), negm);
+          const float p0 = ex2(f2_lo(x)), p1 = ex2(f2_hi(x));
+          r4[i & 3] = f2_add(r4[i & 3], f2(p0, p1));
           pk[i] = pack_bf16(p0, p1);
         }
         tc::tmem_st16(tmem + lane_base + scol + (uint32_t)(q * 16), pk);
       }
       tc::tmem_st_wait();
-      l += ((r8[0] + r8[1]) + (r8[2] + r8[3])) + ((r8[4] + r8[5]) + (r8[6] + r8[7]));
+      {
+        const uint64_t r2 = f2_add(f2_add(r4[0], r4[1]), f2_add(r4[2], r4[3]));
+        l += f2_lo(r2) + f2_hi(r2);
+      }
       tc::tc_fence_before();
       tc::mbar_arrive(p_full + t);
     }
