@@ -46,6 +46,9 @@ def _args():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--heads", type=int, default=None,
                     help="run only the first H heads of the workload (small profiler captures)")
+    ap.add_argument("--shard-heads", action="store_true",
+                    help="split one layer's heads over the ranks and all-gather O (strong scaling); "
+                         "the default runs one whole layer per rank (weak scaling)")
     ap.add_argument("--stress", action="store_true",
                     help="error against dense attention over the noise sigma x budget rho grid "
                          "of the stress workload, for the method's router and two ablations")
@@ -170,48 +173,74 @@ def attn_traffic(cfg):
 
 # ----------------------------------------------------------------- oracle
 
-def oracle_sample(cfg, rho, q, k, v, iq, ik):
-    """Time the CPU oracle on a bounded sample of one head and extrapolate to
-    the whole layer.  Returns (seconds per layer, description, threads)."""
+def _stratified(lq, C, n):
+    """About n query rows spread over the query clusters: the first
+    ceil(n / C) members of every non-empty cluster."""
+    import numpy as np
+    per = -(-n // C)
+    return np.sort(np.concatenate([np.nonzero(lq == a)[0][:per] for a in range(C)]))
+
+
+def oracle_sample(cfg, rho, q, k, v, iq, ik, key_frac=1, rows=1024):
+    """Time the CPU oracle (float32 NumPy, multithreaded BLAS) on a bounded
+    sample of one head and extrapolate to the whole layer: one k-means round
+    of Q and of K (x iters), the final assignment, the permutation and value
+    centroids, the block error on `key_frac` of the keys (all by default;
+    scaled by 1 / key_frac), the routing, and the hybrid attention on `rows`
+    query rows spread over the query clusters (scaled by N / rows); times H.
+    Returns (extrapolated seconds per layer, description, stage seconds,
+    measured seconds of the sample)."""
     import numpy as np
     from oracle import svgear_oracle as ora
     s = 1.0 / math.sqrt(cfg.d)
     t = {}
-    t0 = time.perf_counter()
-    lab_q = ora.assign(q, iq); mu_q, _ = ora.update(q, lab_q, iq)
-    t["kmeans_q_iter"] = time.perf_counter() - t0
-    t0 = time.perf_counter()
-    lab_k = ora.assign(k, ik); mu_k, _ = ora.update(k, lab_k, ik)
-    t["kmeans_k_iter"] = time.perf_counter() - t0
-    t0 = time.perf_counter()
-    lq = ora.assign(q, mu_q); lk = ora.assign(k, mu_k)
-    t["final_assign"] = time.perf_counter() - t0
-    t0 = time.perf_counter()
-    pq, oq, cq = ora.permute(lq, cfg.Cq); pk, ok, ck = ora.permute(lk, cfg.Ck)
-    Vbar = ora.value_centroids(v, lk, cfg.Ck)
-    _ = (q[pq], k[pk], v[pk])
-    t["permute"] = time.perf_counter() - t0
-    frac = 8
-    sub = slice(0, cfg.N // frac)
-    t0 = time.perf_counter()
-    E_part, M = ora.block_error(mu_q, mu_k, Vbar, k[sub], v[sub], lk[sub], ck, s)
-    t["block_error"] = (time.perf_counter() - t0) * frac
-    E = E_part
-    t0 = time.perf_counter()
-    mask, _, _ = ora.route(E, ck, cq, rho)
-    t["route"] = time.perf_counter() - t0
-    rows = np.nonzero(np.isin(lq, np.arange(min(4, cfg.Cq))))[0][:512]
-    lq_s = np.full_like(lq, -1)
-    lq_s[rows] = lq[rows]
-    t0 = time.perf_counter()
-    ora.hybrid_attention(q, k, v, lq_s, lk, mu_k, Vbar, ck, mask, s)
-    t["attn"] = (time.perf_counter() - t0) * (cfg.N / max(1, rows.size))
+    w0 = time.perf_counter()
+    with ora.timing_precision(np.float32):
+        q, k, v, iq, ik = (np.asarray(x, dtype=np.float32) for x in (q, k, v, iq, ik))
+        t0 = time.perf_counter()
+        lab_q = ora.assign(q, iq); mu_q, _ = ora.update(q, lab_q, iq)
+        t["kmeans_q_iter"] = time.perf_counter() - t0
+        t0 = time.perf_counter()
+        lab_k = ora.assign(k, ik); mu_k, _ = ora.update(k, lab_k, ik)
+        t["kmeans_k_iter"] = time.perf_counter() - t0
+        t0 = time.perf_counter()
+        lq = ora.assign(q, mu_q); lk = ora.assign(k, mu_k)
+        t["final_assign"] = time.perf_counter() - t0
+        t0 = time.perf_counter()
+        pq, oq, cq = ora.permute(lq, cfg.Cq); pk, ok, ck = ora.permute(lk, cfg.Ck)
+        Vbar = ora.value_centroids(v, lk, cfg.Ck)
+        _ = (q[pq], k[pk], v[pk])
+        t["permute"] = time.perf_counter() - t0
+        nk = max(1, int(cfg.N * key_frac))
+        t0 = time.perf_counter()
+        E, M = ora.block_error(mu_q, mu_k, Vbar, k[:nk], v[:nk], lk[:nk], ck, s)
+        t["block_error"] = (time.perf_counter() - t0) * cfg.N / nk
+        t0 = time.perf_counter()
+        mask, _, _ = ora.route(E, ck, cq, rho)
+        t["route"] = time.perf_counter() - t0
+        # attention time is linear in the rows plus a per-cluster cost (each
+        # query cluster gathers its routed keys once): time one row per
+        # cluster and the full sample, and extrapolate the line to N rows
+        ta = []
+        for n_rows in (cfg.Cq, rows):
+            r = _stratified(lq, cfg.Cq, n_rows)
+            lq_s = np.full_like(lq, -1)
+            lq_s[r] = lq[r]
+            t0 = time.perf_counter()
+            ora.hybrid_attention(q, k, v, lq_s, lk, mu_k, Vbar, ck, mask, s)
+            ta.append((r.size, time.perf_counter() - t0))
+        (n1, t1), (n2, t2) = ta
+        per_row = max(t2 - t1, 0.0) / max(n2 - n1, 1)
+        t["attn"] = t1 + per_row * (cfg.N - n1)
+    measured = time.perf_counter() - w0
     per_head = (cfg.iters * (t["kmeans_q_iter"] + t["kmeans_k_iter"]) + t["final_assign"]
                 + t["permute"] + t["block_error"] + t["route"] + t["attn"])
-    desc = (f"oracle (float64 NumPy) on head 0: one k-means round of Q and K timed and x{cfg.iters}, "
-            f"final assignment, permutation, block error on 1/{frac} of the keys (x{frac}), routing, "
-            f"hybrid attention on {rows.size} query rows (x N/rows); extrapolated to {cfg.H} heads")
-    return per_head * cfg.H, desc, t
+    keys = "all keys" if nk == cfg.N else f"{nk} of {cfg.N} keys (x{cfg.N / nk:.2f})"
+    desc = (f"oracle in float32 NumPy on head 0 ({measured:.1f} s measured): one k-means round of Q and "
+            f"of K timed and x{cfg.iters}, final assignment, permutation and value centroids, block "
+            f"error on {keys}, routing, hybrid attention on {n1} and on {n2} query rows spread over the "
+            f"{cfg.Cq} query clusters (time extrapolated linearly to N rows); x {cfg.H} heads")
+    return per_head * cfg.H, desc, t, measured
 
 
 def _threads():
@@ -245,30 +274,117 @@ def job_value(cfg, world, ms):
 
 
 def run_reference(a, cfg, rho):
+    """The reference arm: the CPU oracle (float32 NumPy, the machine's host
+    cores) on a bounded sample of the same workload per step, extrapolated
+    to the layer.  The sample is sized so that warm-up + timed steps end
+    within about three minutes; the line reports the measured sample time per
+    step beside the extrapolated layer time."""
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return 0
-    import numpy as np
     from clustered_sparse_attention_flash_b200 import synth
     q, k, v, _ = synth.make_head(cfg, 0)
     iq = synth.forgy_init(cfg, q, 0, 0, cfg.Cq)
     ik = synth.forgy_init(cfg, k, 0, 1, cfg.Ck)
-    secs = []
-    for i in range(a.warmup + a.steps):
-        t0 = time.perf_counter()
-        est, desc, _ = oracle_sample(cfg, rho, q, k, v, iq, ik)
+    n = a.warmup + a.steps
+    # full sample (all keys, 1,024 rows) when few steps run; a quarter of the
+    # keys and 256 rows per step otherwise
+    key_frac, rows = (1, 1024) if n <= 6 else (0.25, 256)
+    est_s, meas_s = [], []
+    for i in range(n):
+        est, desc, _, meas = oracle_sample(cfg, rho, q, k, v, iq, ik, key_frac=key_frac, rows=rows)
         if i >= a.warmup:
-            secs.append(est)
-    layer_s = statistics.mean(secs)
+            est_s.append(est)
+            meas_s.append(meas)
+    layer_s = statistics.mean(est_s)
     val = dense_flops(cfg) / layer_s / 1e12
     line = {"impl": "reference", "metric": METRIC, "value": val, "unit": UNIT, "n_gpus": a.gpus,
             "steps": a.steps, "warmup": a.warmup, "ms_per_step": layer_s * 1e3,
-            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "ms_per_step_basis": "extrapolated: each step times a bounded sample of one head and scales "
+                                 "it to the whole layer (see cpu_baseline.sample)",
+            "sample_ms_per_step_measured": statistics.mean(meas_s) * 1e3,
+            "steps_timed": len(meas_s),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
             "data": "synthetic", "config": {"workload": _workload(cfg, rho)},
             "cpu_baseline": {"value": val, "unit": UNIT, "cores": _threads(), "kind": "oracle",
-                             "sample": desc},
+                             "sample": desc, "extrapolated": True},
             "e2e": {"value": val, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
+    return 0
+
+
+# ----------------------------------------------------------- head sharding
+
+def run_shard_heads(a, cfg, rho):
+    """One layer of cfg split by heads over the ranks (strong scaling): rank r
+    runs heads head_range(H, world, r) through svgear_forward, then one NCCL
+    all-gather assembles O [H, N, d] on every rank.  Both are inside the timed
+    region; the time is the slowest rank's."""
+    q_np, k_np, v_np, iq_np, ik_np = generate(cfg)   # before any CUDA call
+    import torch
+    from clustered_sparse_attention_flash_b200 import svgear as sv
+    from clustered_sparse_attention_flash_b200.shard import forward_heads_sharded, head_range
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dist = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=600))
+    try:
+        dev = torch.device("cuda", local)
+        tdt = torch.bfloat16 if cfg.dtype == "bf16" else torch.float32
+        dQ, dK, dV = (torch.from_numpy(x).to(tdt).to(dev) for x in (q_np, k_np, v_np))
+        iq, ik = torch.from_numpy(iq_np).to(dev), torch.from_numpy(ik_np).to(dev)
+        s = 1.0 / math.sqrt(cfg.d)
+        b, e = head_range(cfg.H, world, rank)
+        p = sv.params(e - b, cfg.N, cfg.N, cfg.d, cfg.Cq, cfg.Ck, cfg.iters, rho, s,
+                      sv.SVGEAR_BF16 if cfg.dtype == "bf16" else sv.SVGEAR_F32)
+        ws = sv.workspace(sv.svgear_workspace_size(p), dev)
+        stream = torch.cuda.current_stream(dev)
+
+        def compute(q, k, v, Cq, Ck, iters, r, sc, iq_, ik_):
+            O = torch.empty_like(q)
+            sv.svgear_forward(q, k, v, p, iq_, ik_, O, ws, ws.numel(), stream)
+            return O
+
+        def step():
+            return forward_heads_sharded(dQ, dK, dV, cfg.Cq, cfg.Ck, cfg.iters, rho, s, iq, ik,
+                                         compute=compute)[0]
+
+        for _ in range(a.warmup):
+            step()
+        torch.cuda.synchronize(dev)
+        assert sv.svgear_get_status(stream) == sv.SVGEAR_OK
+        if dist is not None:
+            dist.barrier()
+        torch.cuda.synchronize(dev)
+        ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        l0 = sv.svgear_launch_count()
+        ev0.record(stream)
+        for _ in range(a.steps):
+            step()
+        ev1.record(stream)
+        torch.cuda.synchronize(dev)
+        launches = sv.svgear_launch_count() - l0
+        if dist is not None:
+            dist.barrier()
+        ms = max_over_ranks(ev0.elapsed_time(ev1) / a.steps, dist, dev)
+        if rank == 0:
+            line = {"metric": METRIC, "value": dense_flops(cfg) / (ms / 1e3) / 1e12, "unit": UNIT,
+                    "n_gpus": world, "steps": a.steps, "warmup": a.warmup, "ms_per_step": ms,
+                    "higher_is_better": True, "scaling": "strong", "vs_baseline": None, "dtype": cfg.dtype,
+                    "data": "synthetic",
+                    "config": {"workload": _workload(cfg, rho),
+                               "parallelism": f"heads sharded x{world} ({e - b} heads on rank 0), "
+                                              f"all-gather of O over the process group"},
+                    "gpu_launches": launches}
+            print(json.dumps(line), flush=True)
+    finally:
+        if dist is not None:
+            dist.destroy_process_group()
     return 0
 
 
@@ -380,6 +496,8 @@ def main():
     rho = cfg.rho if a.rho is None else a.rho
     if a.impl == "reference":
         return run_reference(a, cfg, rho)
+    if a.shard_heads:
+        return run_shard_heads(a, cfg, rho)
     assert a.warmup >= 3, "at least 3 warm-up steps"
 
     q_np, k_np, v_np, iq_np, ik_np = generate(cfg)   # before any CUDA call
@@ -517,9 +635,10 @@ def main():
 
     cpu = None
     if rank == 0 and world == 1 and not a.no_cpu_baseline:
-        sec, desc, _ = oracle_sample(cfg, rho, q_np[0], k_np[0], v_np[0], iq_np[0], ik_np[0])
+        sec, desc, stages, meas = oracle_sample(cfg, rho, q_np[0], k_np[0], v_np[0], iq_np[0], ik_np[0])
         cpu = {"value": dense_flops(cfg) / sec / 1e12, "unit": UNIT, "cores": _threads(),
-               "kind": "oracle", "sample": desc, "layer_s_extrapolated": sec}
+               "kind": "oracle", "sample": desc, "extrapolated": True, "layer_s_extrapolated": sec,
+               "sample_s_measured": meas, "stage_s_per_head": stages}
 
     value = job_value(cfg, world, ms)
     line = {

@@ -151,6 +151,12 @@ int svgear_get_status(void* stream) {
   return SVGEAR_ERR_INVALID;
 }
 
+int svgear_selftest_wait(long long limit_ns, void* stream) {
+  if (limit_ns < 1000 || limit_ns > 1000000000LL) return SVGEAR_ERR_INVALID;
+  if (!status_word()) return SVGEAR_ERR_CUDA;
+  return cuda_status(selftest_wait_run((uint64_t)limit_ns, S(stream)));
+}
+
 size_t svgear_kmeans_workspace_size(int H, int N, int d, int C) {
   if (check_shape(H, N, d, C, SVGEAR_F32)) return 0;
   return kmeans_ws_bytes(H, N, d, C);

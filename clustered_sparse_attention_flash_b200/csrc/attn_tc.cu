@@ -563,6 +563,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           t = pos - pos0;
         }
+        // the window must be covered up to the stream end (status word if not)
+        if (lane == 0 && (long long)t < min((long long)BN, lex - pos0)) set_status(status, ST_BOUNDS);
         npc = __shfl_sync(0xffffffffu, npc, 0);
         tail = __shfl_sync(0xffffffffu, t, 0);
         bytes = (uint32_t)__shfl_sync(0xffffffffu, nb, 0) * kGroup;

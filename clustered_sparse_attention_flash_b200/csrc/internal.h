@@ -15,6 +15,10 @@ int* status_word();
 // Counts kernel launches issued by the library (svgear_launch_count).
 void note_launch();
 
+// Self-test of the bounded in-kernel waits: one block whose wait on a barrier
+// that nothing completes gives up after limit_ns (ST_TIMEOUT).
+cudaError_t selftest_wait_run(uint64_t limit_ns, cudaStream_t st);
+
 // Host-side validation of an operator parameter block (svgear_status code).
 int params_status(const svgear_params* p);
 

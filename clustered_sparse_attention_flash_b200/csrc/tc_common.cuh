@@ -59,17 +59,18 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
 
 // Waits until the phase with parity `parity` of `bar` completed.  Gives up
-// when `abort_flag` is raised by another role or after kWaitLimitNs, in which
-// case it records ST_TIMEOUT, raises the abort flag and returns false.
+// when `abort_flag` is raised by another role or after `limit_ns` (kWaitLimitNs
+// unless a caller asks for less), in which case it records ST_TIMEOUT, raises
+// the abort flag and returns false.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
-                                          int* status) {
+                                          int* status, uint64_t limit_ns = kWaitLimitNs) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer();
   for (uint32_t it = 1;; ++it) {
     if (mbar_try_wait(bar, parity)) return true;
     if ((it & 255u) == 0) {
       if (*abort_flag) return false;
-      if (globaltimer() - t0 > kWaitLimitNs) {
+      if (globaltimer() - t0 > limit_ns) {
         set_status(status, ST_TIMEOUT);
         *abort_flag = 1;
         return false;
@@ -88,8 +89,8 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t by
 // instructions: the result is made uniform across the warp, so that either
 // every lane goes on or every lane takes the abort path.
 __device__ __forceinline__ bool mbar_wait_warp(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
-                                               int* status) {
-  const bool ok = mbar_wait(bar, parity, abort_flag, status);
+                                               int* status, uint64_t limit_ns = kWaitLimitNs) {
+  const bool ok = mbar_wait(bar, parity, abort_flag, status, limit_ns);
   return __all_sync(0xffffffffu, ok);
 }
 

@@ -75,6 +75,7 @@ _SIGS = {
     "svgear_status_string": (ctypes.c_char_p, [_I]),
     "svgear_launch_count": (ctypes.c_longlong, []),
     "svgear_get_status": (_I, [_P]),
+    "svgear_selftest_wait": (_I, [ctypes.c_longlong, _P]),
     "svgear_kmeans_workspace_size": (_SZ, [_I, _I, _I, _I]),
     "svgear_kmeans": (_I, [_P, _I, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P, _SZ, _P]),
     "svgear_permute_workspace_size": (_SZ, [_I, _I, _I]),
@@ -168,6 +169,10 @@ svgear_status_string = status_string
 
 def svgear_get_status(stream=None) -> int:
     return lib().svgear_get_status(_stream(stream))
+
+
+def svgear_selftest_wait(limit_ns: int, stream=None) -> None:
+    _check("svgear_selftest_wait", lib().svgear_selftest_wait(int(limit_ns), _stream(stream)))
 
 
 def svgear_kmeans_workspace_size(H, N, d, C) -> int:

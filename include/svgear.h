@@ -33,6 +33,11 @@
  *    and timed-out waits inside kernels are recorded in a device status word
  *    that svgear_get_status reads.
  *  - No exceptions or aborts cross the ABI.
+ *  - The library looks up the device addresses of its own device variables
+ *    (the status word; the scratch array of svgear_block_error_noalloc) once
+ *    per device and keeps them for the life of the process.  After a
+ *    cudaDeviceReset the module is loaded again at new addresses, so a
+ *    process that resets a device must not call the library on it again.
  */
 #ifndef SVGEAR_H
 #define SVGEAR_H
@@ -144,6 +149,16 @@ SVGEAR_API const char* svgear_status_string(int status);
  * itself failed (a sticky CUDA error). */
 SVGEAR_API int svgear_get_status(void* stream);
 
+/* Self-test of the failure detection (no counterpart in the pages): enqueues
+ * on `stream` one block that waits on an mbarrier nothing ever completes,
+ * with the wait routine and the abort protocol of the operator's tensor-core
+ * kernels but a limit of `limit_ns` nanoseconds (1e3 .. 1e9; other values
+ * return SVGEAR_ERR_INVALID).  The wait gives up, the block releases its
+ * tensor memory and ends, and the next svgear_get_status returns
+ * SVGEAR_ERR_TIMEOUT; the context stays usable.  No device memory is
+ * allocated and nothing else is touched. */
+SVGEAR_API int svgear_selftest_wait(long long limit_ns, void* stream);
+
 /* ---------------------------------------------------------------------------
  * (1) k-means (Lloyd) on X [H,N,d] with C clusters.  Review step (1), "Flash
  * k-means" clustering of queries and keys; gist.science summary 2.A.
@@ -222,7 +237,8 @@ SVGEAR_API int svgear_block_error(const float* Qbar, const float* Kbar, const fl
  *     SVGEAR_ERR_WORKSPACE without enqueuing anything;
  *   - the first call on a device looks up the array's device address
  *     (cudaGetSymbolAddress) with that device current; make that first call
- *     before any stream capture;
+ *     before any stream capture.  The address is kept for the process, so
+ *     the entry must not be called again on a device after cudaDeviceReset;
  *   - every call shares the one array, so calls that overlap on the GPU
  *     (different streams, or different host threads on one device) race and
  *     must be ordered by the caller.  Each call writes the scratch fully

@@ -43,6 +43,11 @@ Readings taken where the pages are silent (each listed in the design notes):
   ranked by the unshifted ratio.
 
 Arrays are per head: X [N, d]; centroids [C, d]; labels [N] ints.
+
+Precision: every function computes in float64.  `timing_precision` lets the
+benchmark's CPU-baseline leg time the same code in float32 (the arithmetic
+and the step order are unchanged, only the element type); parity checks
+never use it.
 """
 from __future__ import annotations
 
@@ -52,10 +57,28 @@ from typing import Dict
 import numpy as np
 
 _ROW_CHUNK = 2048
+_REAL = np.float64
 
 
 def _f64(x) -> np.ndarray:
-    return np.asarray(x, dtype=np.float64)
+    return np.asarray(x, dtype=_REAL)
+
+
+class timing_precision:
+    """Context manager: run the oracle in `dtype` (np.float32 for the CPU
+    timing baseline) instead of float64 inside the `with` block."""
+
+    def __init__(self, dtype):
+        self.dtype = dtype
+
+    def __enter__(self):
+        global _REAL
+        self.old, _REAL = _REAL, self.dtype
+        return self
+
+    def __exit__(self, *exc):
+        global _REAL
+        _REAL = self.old
 
 
 # --------------------------------------------------------------------------
@@ -156,7 +179,7 @@ def value_centroids(V, k_labels, Ck: int) -> np.ndarray:
     [R] steps (2),(4); [AB] "keys and values ... summarized by centroids"."""
     V = _f64(V)
     counts = np.bincount(k_labels, minlength=Ck)
-    sums = np.zeros((Ck, V.shape[1]))
+    sums = np.zeros((Ck, V.shape[1]), dtype=V.dtype)
     np.add.at(sums, k_labels, V)
     out = np.zeros_like(sums)
     nz = counts > 0
@@ -201,7 +224,7 @@ def block_error(Qbar, Kbar, Vbar, K, V, k_labels, k_counts, scale: float,
     k_counts = np.asarray(k_counts)
     M = block_shift(Qbar, Kbar, k_counts, scale)
     Lbar = scale * (Qbar @ Kbar.T)
-    E = np.zeros((Qbar.shape[0], Kbar.shape[0]))
+    E = np.zeros((Qbar.shape[0], Kbar.shape[0]), dtype=K.dtype)
     for s in range(0, K.shape[0], key_chunk):
         j = slice(s, s + key_chunk)
         c = k_labels[j]
@@ -410,7 +433,7 @@ def hybrid_attention(Q, K, V, q_labels, k_labels, Kbar, Vbar, k_counts, mask,
             r = rows[s:s + _ROW_CHUNK]
             L = np.concatenate([scale * (Q[r] @ K[keys].T),
                                 scale * (Q[r] @ Kbar[cc].T)
-                                + np.log(k_counts[cc].astype(np.float64))[None]],
+                                + np.log(k_counts[cc].astype(Q.dtype))[None]],
                                axis=1)
             W = np.exp(L - L.max(axis=1, keepdims=True))
             Vals = np.concatenate([V[keys], Vbar[cc]], axis=0)

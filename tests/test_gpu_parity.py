@@ -9,8 +9,8 @@ import pytest
 
 from clustered_sparse_attention_flash_b200 import svgear as sv
 from oracle import svgear_oracle as ora
-from helpers import (E_FLOOR, E_RTOL, OUT_TOL, TIE_REL, assert_close, case, dev, host,
-                     label_mismatches_are_ties, torch_dtype)
+from helpers import (E_FLOOR, E_RTOL, OUT_TOL, TIE_REL, assert_close, case, check_forward_given_gpu_clusters,
+                     dev, host, label_mismatches_are_ties, stratified_rows, torch_dtype)
 
 torch = pytest.importorskip("torch")
 pytestmark = pytest.mark.gpu
@@ -236,35 +236,34 @@ def test_hybrid_attn_given_oracle_routing(name, rho):
 
 # --------------------------------------------------------------- end to end
 
-@pytest.mark.parametrize("name", CONFIGS)
-def test_forward_end_to_end(name):
-    cs = case(name)
+@pytest.mark.parametrize("name,rho", [("tiny", None), ("mid", None), ("mid", 0.1)])
+def test_forward_end_to_end(name, rho):
+    """Whole forwards: every head is checked stage by stage against the oracle
+    given the GPU's own clusters (never skipped), and, where the ten chained
+    k-means rounds reproduced the oracle's clustering, the block error and the
+    output are also held to the independent oracle run."""
+    cs = case(name, rho=rho)
     cfg = cs.cfg
     O, ws, p, _ = sv.forward(cs.dq(), cs.dk(), cs.dv(), cfg.Cq, cfg.Ck, cfg.iters, cs.rho, cs.scale,
                              dev(cs.init_q), dev(cs.init_k))
     torch.cuda.synchronize()
     assert sv.svgear_get_status() == sv.SVGEAR_OK
     views = sv.view_tensors(p, ws)
+    O = host(O)
+    for i in range(cs.H):
+        check_forward_given_gpu_clusters(views, O[i], i, cs.q[i], cs.k[i], cs.v[i], cfg.Cq, cfg.Ck, cs.rho,
+                                         cs.scale, cfg.dtype)
     lq, lk = host(views["labels_q"]), host(views["labels_k"])
     mask, E = host(views["mask"]), host(views["E"])
-    O = host(O)
     atol, rtol = OUT_TOL[cfg.dtype]
-    strict = 0
     for i in range(cs.H):
         o = cs.oracle[i]
-        kc = host(views["counts_k"])[i]
-        budget = ora.route_budget(cs.rho, cfg.N)
-        assert all((kc * mask[i, a]).sum() <= budget for a in range(cfg.Cq))
         if not (np.array_equal(lq[i], o["q_labels"]) and np.array_equal(lk[i], o["k_labels"])):
-            # clustering diverged at a near-tie somewhere in the 10 chained
-            # rounds; the stage tests above pin every step on identical inputs
-            continue
-        strict += 1
+            continue  # a near-tie moved a label somewhere in the chained rounds
         err = np.abs(E[i] - o["E"])
-        assert (err <= 1e-2 * np.abs(o["E"]) + 1e-5 * np.abs(o["E"]).max()).all()
+        assert (err <= E_RTOL * np.abs(o["E"]) + 1e-6 * np.abs(o["E"]).max()).all()
         if np.array_equal(mask[i], o["mask"]):
             assert_close(O[i], o["O"], atol, rtol, f"forward output head {i}")
-    assert strict >= 1, "no head reproduced the oracle clustering"
 
 
 # -------------------------------------------------------------- edge cases
@@ -285,6 +284,7 @@ def _small(N, d, seed, dtype):
     (300, 64, 4, 300, 0.2),      # singleton key clusters: exact for any rho
     (517, 128, 6, 9, 1.0),       # rho = 1: dense attention
     (130, 64, 1, 2, 0.5),        # one query cluster
+    (257, 128, 3, 5, 0.4),       # a query cluster of more than two 128-row tiles
 ])
 def test_forward_edge_cases(dtype, N, d, Cq, Ck, rho):
     q, k, v = _small(N, d, N + Ck, dtype)
@@ -293,18 +293,36 @@ def test_forward_edge_cases(dtype, N, d, Cq, Ck, rho):
     iq, ik = q[:, :Cq].copy(), k[:, :Ck].copy()
     O, ws, p, _ = sv.forward(dev(q, tdt), dev(k, tdt), dev(v, tdt), Cq, Ck, 4, rho, s, dev(iq), dev(ik))
     torch.cuda.synchronize()
+    assert sv.svgear_get_status() == sv.SVGEAR_OK
     O = host(O)[0]
-    o = ora.forward(q[0], k[0], v[0], Cq, Ck, 4, rho, s, iq[0], ik[0])
-    atol, rtol = OUT_TOL[dtype]
     views = sv.view_tensors(p, ws)
-    same = (np.array_equal(host(views["labels_q"])[0], o["q_labels"])
-            and np.array_equal(host(views["labels_k"])[0], o["k_labels"]))
+    check_forward_given_gpu_clusters(views, O, 0, q[0], k[0], v[0], Cq, Ck, rho, s, dtype)
+    atol, rtol = OUT_TOL[dtype]
     if rho == 1.0 or Ck == N:
         assert_close(O, ora.dense_attention(q[0], k[0], v[0], s), atol, rtol, "dense special case")
     if Ck == 1 and rho == 0.0:
         assert_close(O, np.broadcast_to(v[0].astype(np.float64).mean(0), O.shape), atol, rtol, "mean of V")
-    if same and np.array_equal(host(views["mask"])[0], o["mask"]):
-        assert_close(O, o["O"], atol, rtol, "edge output")
+
+
+@pytest.mark.parametrize("N,Ck,rho", [(8192, 1000, 1.0), (16384, 2000, 0.7)])
+def test_forward_many_routed_clusters(N, Ck, rho):
+    """Query clusters that route more key clusters than the attention kernel
+    stages in shared memory (512): its producers then walk the selection list
+    instead of the staged ranges.  Random bf16 inputs, d = 128."""
+    d, Cq = 128, 8
+    q, k, v = _small(N, d, 7 + Ck, "bf16")
+    s = 1 / math.sqrt(d)
+    iq, ik = q[:, :Cq].copy(), k[:, :Ck].copy()
+    bf = torch.bfloat16
+    O, ws, p, _ = sv.forward(dev(q, bf), dev(k, bf), dev(v, bf), Cq, Ck, 3, rho, s, dev(iq), dev(ik))
+    torch.cuda.synchronize()
+    assert sv.svgear_get_status() == sv.SVGEAR_OK
+    views = sv.view_tensors(p, ws)
+    nsel = host(views["n_sel"])[0]
+    assert nsel.max() > 512, nsel.max()
+    lq = host(views["labels_q"])[0]
+    rows = stratified_rows(lq, Cq, 512, np.random.default_rng(Ck))
+    check_forward_given_gpu_clusters(views, host(O)[0], 0, q[0], k[0], v[0], Cq, Ck, rho, s, "bf16", rows=rows)
 
 
 def test_forward_empty_key_cluster():
@@ -346,3 +364,19 @@ def test_kmeans_assign_wide(N, d, C, seed):
     nd = label_mismatches_are_ties(X, mu, lab[0])
     assert nd <= 2, nd
     np.testing.assert_array_equal(cnt[0], np.bincount(lab[0], minlength=C))
+
+
+def test_head_sharded_forward_one_rank_is_the_forward():
+    """The head-sharded entry with a single process runs every head through
+    svgear_forward and returns exactly the plain forward's output."""
+    from clustered_sparse_attention_flash_b200.shard import forward_heads_sharded
+    cs = case("mid")
+    cfg = cs.cfg
+    O1, _, _, _ = sv.forward(cs.dq(), cs.dk(), cs.dv(), cfg.Cq, cfg.Ck, cfg.iters, cs.rho, cs.scale,
+                             dev(cs.init_q), dev(cs.init_k))
+    O2, hr = forward_heads_sharded(cs.dq(), cs.dk(), cs.dv(), cfg.Cq, cfg.Ck, cfg.iters, cs.rho, cs.scale,
+                                   dev(cs.init_q), dev(cs.init_k))
+    torch.cuda.synchronize()
+    assert sv.svgear_get_status() == sv.SVGEAR_OK
+    assert hr == (0, cs.H)
+    assert torch.equal(O1, O2)
