@@ -68,8 +68,8 @@ constexpr int kUnitRows = 2 * BQ;  // query rows of one block
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr uint32_t kColS = 0, kColO = 256;
 constexpr int kMaxRanges = 512;  // routed clusters staged in shared memory
-constexpr int kRegsLow = 56;     // MMA / producer warpgroup after the split
-constexpr int kRegsHigh = 208;   // each softmax warpgroup after the split
+constexpr int kRegsLow = 48;     // MMA / producer warpgroup after the split
+constexpr int kRegsHigh = 224;   // each softmax warpgroup after the split
 // the split fits a launch of 168 registers per thread (checked at launch)
 static_assert(4 * 32 * kRegsLow + 8 * 32 * kRegsHigh <= kThreads * 168, "register split");
 
@@ -258,7 +258,8 @@ struct AttnSmem {
   static constexpr int k_off = q_off + 2 * kQTile;                   // [kKSlots] key tiles
   static constexpr int v_off = k_off + kKSlots * kKTile;             // [kVSlots] value tiles
   static constexpr int bias_off = v_off + kVSlots * kKTile;          // [kBSlots][BN] log2 biases
-  static constexpr int bits_off = bias_off + kBSlots * BN * 4;
+  static constexpr int nv_off = bias_off + kBSlots * BN * 4;         // [kBSlots] valid keys of the stage
+  static constexpr int bits_off = nv_off + 16;
   static constexpr int rng_off = bits_off + kMaxCkBits / 8;          // [3][kMaxRanges] start, prefix, len
   static constexpr int pc_off = rng_off + 3 * kMaxRanges * 4 + 16;   // [producer warp][32] piece lists
   static constexpr int bar_off = pc_off + 2 * 32 * 16;
@@ -287,6 +288,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   float* bias_s = reinterpret_cast<float*>(smem + S::bias_off);
+  int* nv_s = reinterpret_cast<int*>(smem + S::nv_off);
   uint32_t* bits = reinterpret_cast<uint32_t*>(smem + S::bits_off);
   int* rng_start = reinterpret_cast<int*>(smem + S::rng_off);  // first padded row of routed range i
   int* rng_cum = rng_start + kMaxRanges;                        // padded rows in ranges [0, i)
@@ -637,10 +639,13 @@ __global__ void __launch_bounds__(kThreads, 1)
           // valid keys 0, padding and the stream tail -inf
           for (int i = lane; i < BN; i += 32) bias[i] = -INFINITY;
           __syncwarp();
+          int nvalid = 0;
           for (int q = 0; q < npc; ++q) {
             const int4 pc = pcs[q];
             for (int i = lane; i < pc.w; i += 32) bias[pc.x * 8 + i] = 0.f;
+            nvalid += pc.w;
           }
+          if (lane == 0) nv_s[sb] = nvalid;
         } else if (p == 0) {
           const int c0 = (j - n_ex) * BN;
           for (int i = lane; i < BN; i += 32) {
@@ -705,32 +710,54 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc::tmem_ld32(tmem + lane_base + scol + 64u, *reinterpret_cast<uint32_t(*)[32]>(v + 64));
       tc::tmem_ld32(tmem + lane_base + scol + 96u, *reinterpret_cast<uint32_t(*)[32]>(v + 96));
       tc::tmem_ld_wait();
+      // Routed stage, fast path: padding and tail keys have zero key rows, so
+      // their logits are exactly 0 and their value rows are 0.  When the raw
+      // maximum of the stage is positive it is a real key's, the scale and
+      // the row maximum are applied in one FMA in the exponential pass, and
+      // the padding's known share is taken off the row sum.  Otherwise (and
+      // for compensation stages) x = s * scale2 + bias with the stage's bias.
+      const uint64_t sc2 = f2(scale2, scale2);
       float mx;
+      bool raw = false;
       {
-        const uint64_t sc2 = f2(scale2, scale2);
         float m8[8];
+        if (j < n_ex) {
 #pragma unroll
-        for (int k = 0; k < 8; ++k) m8[k] = -INFINITY;
+          for (int k = 0; k < 8; ++k) m8[k] = -INFINITY;
 #pragma unroll
-        for (int i = 0; i < 128; i += 16) {
-          const float4 b0 = *reinterpret_cast<const float4*>(bias + i);
-          const float4 b1 = *reinterpret_cast<const float4*>(bias + i + 4);
-          const float4 b2 = *reinterpret_cast<const float4*>(bias + i + 8);
-          const float4 b3 = *reinterpret_cast<const float4*>(bias + i + 12);
-          const float bb[16] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w,
-                                b2.x, b2.y, b2.z, b2.w, b3.x, b3.y, b3.z, b3.w};
+          for (int i = 0; i < 128; i += 16)
 #pragma unroll
-          for (int k = 0; k < 8; ++k) {
-            // x = s * scale2 + bias for two keys per instruction
-            const uint64_t x = f2_fma(f2(__uint_as_float(v[i + 2 * k]), __uint_as_float(v[i + 2 * k + 1])), sc2,
-                                      f2(bb[2 * k], bb[2 * k + 1]));
-            v[i + 2 * k] = __float_as_uint(f2_lo(x));
-            v[i + 2 * k + 1] = __float_as_uint(f2_hi(x));
-            m8[k] = tc::fmax3(m8[k], f2_lo(x), f2_hi(x));
-          }
+            for (int k = 0; k < 8; ++k)
+              m8[k] = tc::fmax3(m8[k], __uint_as_float(v[i + 2 * k]), __uint_as_float(v[i + 2 * k + 1]));
+          const float mr = fmaxf(tc::fmax3(m8[0], m8[1], m8[2]), tc::fmax3(tc::fmax3(m8[3], m8[4], m8[5]), m8[6], m8[7]));
+          raw = __all_sync(0xffffffffu, mr > 0.f);
+          mx = mr * scale2;
         }
-        mx = fmaxf(tc::fmax3(m8[0], m8[1], m8[2]), tc::fmax3(tc::fmax3(m8[3], m8[4], m8[5]), m8[6], m8[7]));
+        if (!raw) {
+#pragma unroll
+          for (int k = 0; k < 8; ++k) m8[k] = -INFINITY;
+#pragma unroll
+          for (int i = 0; i < 128; i += 16) {
+            const float4 b0 = *reinterpret_cast<const float4*>(bias + i);
+            const float4 b1 = *reinterpret_cast<const float4*>(bias + i + 4);
+            const float4 b2 = *reinterpret_cast<const float4*>(bias + i + 8);
+            const float4 b3 = *reinterpret_cast<const float4*>(bias + i + 12);
+            const float bb[16] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w,
+                                  b2.x, b2.y, b2.z, b2.w, b3.x, b3.y, b3.z, b3.w};
+#pragma unroll
+            for (int k = 0; k < 8; ++k) {
+              // x = s * scale2 + bias for two keys per instruction
+              const uint64_t x = f2_fma(f2(__uint_as_float(v[i + 2 * k]), __uint_as_float(v[i + 2 * k + 1])), sc2,
+                                        f2(bb[2 * k], bb[2 * k + 1]));
+              v[i + 2 * k] = __float_as_uint(f2_lo(x));
+              v[i + 2 * k + 1] = __float_as_uint(f2_hi(x));
+              m8[k] = tc::fmax3(m8[k], f2_lo(x), f2_hi(x));
+            }
+          }
+          mx = fmaxf(tc::fmax3(m8[0], m8[1], m8[2]), tc::fmax3(tc::fmax3(m8[3], m8[4], m8[5]), m8[6], m8[7]));
+        }
       }
+      const int npad = raw ? BN - nv_s[sb] : 0;
       // the bias is read: release the stage's bias slot(s) on this warp's behalf
       __syncwarp();
       if (lane == 0)
@@ -760,9 +787,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (grow) m_used = mx;
       const float mref = m_used == -INFINITY ? 0.f : m_used;
       // P = 2^(x - m) in bf16 over the first 64 columns of S[t] (keys 2c and
-      // 2c + 1 in column c; every S value of the row is already in registers)
-      // (x - m for two keys per instruction; row sums in four packed pairs)
+      // 2c + 1 in column c; every S value of the row is already in registers);
+      // x - m (fast path: s * scale2 - m) for two keys per instruction, row
+      // sums in four packed pairs
+      // (fallback: the stored x times 1 minus m, which is x - m exactly)
       const uint64_t negm = f2(-mref, -mref);
+      const uint64_t mul2 = raw ? sc2 : f2(1.f, 1.f);
       uint64_t r4[4] = {0ull, 0ull, 0ull, 0ull};
 #pragma unroll
       for (int q = 0; q < 4; ++q) {
@@ -770,7 +800,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
           const int c = q * 32 + 2 * i;
-          const uint64_t x = f2_add(f2(__uint_as_float(v[c]), __uint_as_float(v[c + 1])), negm);
+          const uint64_t x = f2_fma(f2(__uint_as_float(v[c]), __uint_as_float(v[c + 1])), mul2, negm);
           const float p0 = ex2(f2_lo(x)), p1 = ex2(f2_hi(x));
           r4[i & 3] = f2_add(r4[i & 3], f2(p0, p1));
           pk[i] = pack_bf16(p0, p1);
@@ -780,7 +810,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc::tmem_st_wait();
       {
         const uint64_t r2 = f2_add(f2_add(r4[0], r4[1]), f2_add(r4[2], r4[3]));
-        l += f2_lo(r2) + f2_hi(r2);
+        // the padding keys (fast path) each added 2^(0 - m)
+        l += (f2_lo(r2) + f2_hi(r2)) - (float)npad * ex2(-mref);
       }
       tc::tc_fence_before();
       tc::mbar_arrive(p_full + t);

@@ -95,14 +95,22 @@ __global__ void __launch_bounds__(256) k_update(const T* __restrict__ X, const i
       }
     }
   }
-  for (; r < end; r += NW) {
-    const int i = ph[r];
-    if constexpr (PER == 4) {
-      float4 v = ld4(Xh + (size_t)i * D);
-      acc[0] += v.x; acc[1] += v.y; acc[2] += v.z; acc[3] += v.w;
-    } else {
-      float2 v = ld2(Xh + (size_t)i * D);
-      acc[0] += v.x; acc[1] += v.y;
+  // at most eight rows of this warp remain: one predicated batch (loads in
+  // flight together), added in the same row order as before
+  {
+    int idx[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) idx[u] = r + u * NW < end ? ph[r + u * NW] : -1;
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      if (idx[u] < 0) continue;
+      if constexpr (PER == 4) {
+        float4 v = ld4(Xh + (size_t)idx[u] * D);
+        acc[0] += v.x; acc[1] += v.y; acc[2] += v.z; acc[3] += v.w;
+      } else {
+        float2 v = ld2(Xh + (size_t)idx[u] * D);
+        acc[0] += v.x; acc[1] += v.y;
+      }
     }
   }
 #pragma unroll

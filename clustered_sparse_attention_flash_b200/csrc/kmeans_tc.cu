@@ -394,8 +394,13 @@ __device__ __forceinline__ void consume(const uint32_t (&v)[NV], const int4* __r
 #pragma unroll
   for (int q = 0; q < NV; q += 2) {
     const int4 e = tp[q >> 1];  // {||mu||^2/2, index} of two columns
-    const float s0 = __uint_as_float(v[q]) - __int_as_float(e.x);
-    const float s1 = __uint_as_float(v[q + 1]) - __int_as_float(e.z);
+    // both scores x.mu - ||mu||^2/2 in one two-wide subtraction
+    uint64_t a2, n2, d2;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(a2) : "r"(v[q]), "r"(v[q + 1]));
+    asm("mov.b64 %0, {%1, %2};" : "=l"(n2) : "r"(e.x), "r"(e.z));
+    asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(d2) : "l"(a2), "l"(n2));
+    float s0, s1;
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(s0), "=f"(s1) : "l"(d2));
     const float p0 = __uint_as_float((__float_as_uint(s0) & keep) | (uint32_t)e.y);
     const float p1 = __uint_as_float((__float_as_uint(s1) & keep) | (uint32_t)e.w);
     top3_add2(b1, b2, b3, p0, p1);
