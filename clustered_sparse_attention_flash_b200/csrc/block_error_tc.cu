@@ -12,9 +12,12 @@
 //
 // A block owns whole key clusters (the clusters whose first key falls in its
 // share of the head's keys), so every E[a][c] is one thread's sum in a fixed
-// order.  Block of 6 warps: warp 0 allocates tensor memory and issues MMAs,
-// warp 1 issues the TMA copies of the key tiles and stages the per-key
-// scalars, warps 2-5 are the epilogue (one TMEM lane = one query cluster).
+// order.  Warp 0 allocates tensor memory and issues MMAs, warp 1 issues the
+// TMA copies of the key tiles and stages the per-key scalars, and the
+// remaining warps are kBeGroups epilogue warpgroups (one TMEM lane = one query
+// cluster): group g owns the key clusters c with c % kBeGroups == g and reads
+// only the 32-key chunks of each tile that hold its clusters' keys, so a
+// cluster is still summed by one thread in key order.
 // For the value-agnostic ablation the staged scalars are (0, 0, 1), so each
 // key adds w^2 = (A - B_j)^2 / A^2.
 #include <cuda.h>
@@ -28,7 +31,8 @@ namespace svg {
 
 namespace {
 
-constexpr int kBeThreads = 192;
+constexpr int kBeGroups = 3;                    // epilogue warpgroups (clusters round-robin)
+constexpr int kBeThreads = 64 + 128 * kBeGroups;
 constexpr int kBeKeys = 256;    // keys per tile (MMA N)
 constexpr int kBeStages = 2;
 constexpr int kBeRows = 128;    // query-cluster rows of the A operand (MMA M)
@@ -128,11 +132,11 @@ __global__ void __launch_bounds__(kBeThreads, 1)
     tc::mbar_init(q_full, 1);
     for (int i = 0; i < kBeStages; ++i) {
       tc::mbar_init(full + i, 2);    // TMA arrival with bytes + the scalars' arrival
-      tc::mbar_init(empty + i, 5);   // MMA commit + 4 epilogue warps
+      tc::mbar_init(empty + i, 1 + 4 * kBeGroups);   // MMA commit + every epilogue warp
     }
     for (int i = 0; i < 2; ++i) {
       tc::mbar_init(acc_full + i, 1);
-      tc::mbar_init(acc_empty + i, 4);
+      tc::mbar_init(acc_empty + i, 4 * kBeGroups);
     }
     tc::mbar_init(done, 1);
     *abort_flag = 0;
@@ -198,9 +202,19 @@ __global__ void __launch_bounds__(kBeThreads, 1)
       const float* ks1 = value_agnostic ? nullptr : ks + (size_t)h * Nk;
       for (int t = 0; t < ntiles; ++t) {
         const int s = t % kBeStages;
+        const int j0 = kb + t * kBeKeys;
+        // the tile's per-key scalars go to registers first (all loads in
+        // flight together, before the wait for the stage)
+        float4 vv[kBeKeys / 32];
+#pragma unroll
+        for (int u = 0; u < kBeKeys / 32; ++u) {
+          const int j = j0 + u * 32 + lane;
+          vv[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+          if (j < ke)
+            vv[u] = ks1 ? make_float4(ks1[j], ks1[plane + j], ks1[2 * plane + j], 0.f) : make_float4(0.f, 0.f, 1.f, 0.f);
+        }
         const bool ok = tc::mbar_wait_warp(empty + s, ((t / kBeStages) & 1) ^ 1, abort_flag, status);
         if (!ok) break;
-        const int j0 = kb + t * kBeKeys;
         if (lane == 0) {
           const uint32_t ka = tc::smem_u32(k_s + s * kKStage);
           tc::mbar_arrive_expect_tx(full + s, (uint32_t)kKStage);
@@ -208,37 +222,36 @@ __global__ void __launch_bounds__(kBeThreads, 1)
             tc::tma_load_3d(ka + (uint32_t)(kh * kBeKeys * 128), &tmk, kh * 64, j0, h, full + s);
         }
         float4* sc = sc_s + s * kBeKeys;
-        for (int i = lane; i < kBeKeys; i += 32) {
-          const int j = j0 + i;
-          float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-          if (j < ke)
-            v = ks1 ? make_float4(ks1[j], ks1[plane + j], ks1[2 * plane + j], 0.f) : make_float4(0.f, 0.f, 1.f, 0.f);
-          sc[i] = v;
-        }
+#pragma unroll
+        for (int u = 0; u < kBeKeys / 32; ++u) sc[u * 32 + lane] = vv[u];
         __syncwarp();
         if (lane == 0) tc::mbar_arrive(full + s);
       }
     }
   } else {
     // ------------------------------------------------------------ epilogue
+    const int grp = (warp - 2) >> 2;     // epilogue group: owns clusters c % kBeGroups == grp
     const int quarter = warp & 3;
     const int a = quarter * 32 + lane;   // query cluster == TMEM lane
     const bool act = a < Cq;
     const float Ma = act ? M[(size_t)h * Cq + a] : 0.f;
     const float* La = L + ((size_t)h * Cq + (act ? a : 0)) * Ck;
     float* Ea = E + ((size_t)h * Cq + (act ? a : 0)) * Ck;
-    int c = c_lo, cend = 0, csize = 1;
+    // the group's first cluster at or after c_lo
+    int c = c_lo + ((grp - c_lo % kBeGroups) + kBeGroups) % kBeGroups;
+    int cbeg = 0, cend = 0, csize = 1;
     float Lc = 0.f;
     double acc = 0.0;
-    // moves c to the next non-empty cluster of this block (empty ones get E = 0)
+    // moves c to this group's next non-empty cluster (empty ones get E = 0)
     auto enter = [&]() {
       while (c < c_hi && off[c + 1] == off[c]) {
         if (act) Ea[c] = 0.f;
-        ++c;
+        c += kBeGroups;
       }
       if (c < c_hi) {
+        cbeg = off[c];
         cend = off[c + 1];
-        csize = cend - off[c];
+        csize = cend - cbeg;
         Lc = La[c];
         acc = 0.0;
       }
@@ -248,7 +261,7 @@ __global__ void __launch_bounds__(kBeThreads, 1)
         const float A = expf(Lc - Ma);
         Ea[c] = (float)((double)(A * A) * acc / (double)csize);
       }
-      ++c;
+      c += kBeGroups;
       enter();
     };
     enter();
@@ -265,10 +278,13 @@ __global__ void __launch_bounds__(kBeThreads, 1)
       const int nk = min(kBeKeys, ke - j0);
       const uint32_t base = tc::taddr(tmem, (uint32_t)(quarter * 32), (uint32_t)(buf * kBeKeys));
       for (int q0 = 0; q0 < nk; q0 += 32) {
+        const int k0 = j0 + q0, k1 = j0 + min(q0 + 32, nk);
+        // skip chunks that hold none of this group's keys (block-uniform)
+        if (!(c < c_hi && cbeg < k1)) continue;
         uint32_t v[32];
         tc::tmem_ld32(base + (uint32_t)q0, v);
         tc::tmem_ld_wait();
-        if (q0 + 32 <= nk && j0 + q0 + 32 <= cend) {
+        if (cbeg <= k0 && k0 + 32 <= cend && k1 == k0 + 32) {
           // all 32 keys inside the current cluster (the common case): the
           // terms are independent, with no branch between them
           float t8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
@@ -279,22 +295,25 @@ __global__ void __launch_bounds__(kBeThreads, 1)
             t8[i & 7] += fmaxf(fmaf(w, fmaf(w, e.z, 2.f * e.y), e.x), 0.f);
           }
           acc += (double)(((t8[0] + t8[1]) + (t8[2] + t8[3])) + ((t8[4] + t8[5]) + (t8[6] + t8[7])));
+          if (cend == k1) flush();
           continue;
         }
-        // a cluster boundary or the block's last key inside the chunk
+        // cluster boundaries inside the chunk: walk its keys; keys of other
+        // groups' clusters are passed over (every decision is block-uniform)
         float part = 0.f;
 #pragma unroll
         for (int i = 0; i < 32; ++i) {
-          const int j = j0 + q0 + i;
-          if (j >= ke) break;              // block-uniform
-          if (j >= cend) {                 // block-uniform: the cluster ends here
+          const int j = k0 + i;
+          if (j >= k1 || !(c < c_hi)) break;
+          if (j < cbeg) continue;          // another group's cluster
+          const float4 e = sc[q0 + i];
+          const float w = neg_expm1(__uint_as_float(v[i]) - Lc);
+          part += fmaxf(fmaf(w, fmaf(w, e.z, 2.f * e.y), e.x), 0.f);
+          if (j + 1 == cend) {             // the cluster ends here
             acc += (double)part;
             part = 0.f;
             flush();
           }
-          const float4 e = sc[q0 + i];
-          const float w = neg_expm1(__uint_as_float(v[i]) - Lc);
-          part += fmaxf(fmaf(w, fmaf(w, e.z, 2.f * e.y), e.x), 0.f);
         }
         acc += (double)part;
       }
@@ -305,7 +324,9 @@ __global__ void __launch_bounds__(kBeThreads, 1)
         tc::mbar_arrive(empty + s);
       }
     }
-    if (ok && c < c_hi) flush();  // the last cluster, then trailing empty ones
+    // trailing empty clusters of this group (every non-empty one was flushed
+    // when its last key was summed)
+    if (ok) enter();
   }
 
   tc::tc_fence_before();

@@ -24,7 +24,7 @@ int params_status(const svgear_params* p);
 
 // ---- stable counting sort of labels (shared by k-means update and permute)
 // chunk = tokens per scatter chunk; nchunk = ceil(N / chunk)
-constexpr int kSortChunk = 512;
+constexpr int kSortChunk = 2048;
 size_t sort_ws_bytes(int H, int N, int C);
 // Fills counts [H,C], offsets [H,C+1] and (if perm != null) perm [H,N].
 cudaError_t cluster_sort(const int32_t* labels, int H, int N, int C, int32_t* counts,
