@@ -149,11 +149,12 @@ def _peaks():
 
 # DRAM traffic of the attention kernel from one ncu capture (dram__bytes_read.sum
 # + dram__bytes_write.sum of k_attn_tc on the first 4 heads of the Wan-shaped
-# workload: 324.9 MB, i.e. 81.2 MB per head; traffic grows with the heads).  The
-# figure holds only for the kernel sources it was taken on, identified by hash.
-_ATTN_TRAFFIC = {"bytes_per_head": 324.9e6 / 4, "workload": "wan",
+# workload: 278.7 + 67.0 = 345.7 MB, i.e. 86.4 MB per head; traffic grows with
+# the heads).  The figure holds only for the kernel sources it was taken on,
+# identified by hash.
+_ATTN_TRAFFIC = {"bytes_per_head": 345.679e6 / 4, "workload": "wan",
                  "sources": ("attn_tc.cu", "attn_tc.cuh", "tc_common.cuh"),
-                 "sha1": "f7e1b11454368752bc9b16368575da9f2ea41927"}
+                 "sha1": "2afd20e6c97f427c263d1353e6dd02c5b597a914"}
 
 
 def attn_traffic(cfg):

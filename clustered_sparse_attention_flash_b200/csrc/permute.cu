@@ -41,30 +41,24 @@ __global__ void __launch_bounds__(256) k_value_stats(const T* __restrict__ Vp, c
   double acc[PER];
 #pragma unroll
   for (int t = 0; t < PER; ++t) acc[t] = 0.0;
-  int r0 = beg + w;
-  for (; r0 + 3 * NW < end; r0 += 4 * NW) {  // four rows in flight per warp
-    if constexpr (PER == 4) {
-      float4 v[4];
+  // eight rows per warp in flight; each batch is summed in float32 (fixed
+  // pairwise order) and added to the float64 accumulators once
+  for (int r0 = beg + w; r0 < end; r0 += 8 * NW) {
+    float x[8][PER];
 #pragma unroll
-      for (int u = 0; u < 4; ++u) v[u] = ld4(Vh + (size_t)(r0 + u * NW) * D);
-#pragma unroll
-      for (int u = 0; u < 4; ++u) { acc[0] += v[u].x; acc[1] += v[u].y; acc[2] += v[u].z; acc[3] += v[u].w; }
-    } else {
-      float2 v[4];
-#pragma unroll
-      for (int u = 0; u < 4; ++u) v[u] = ld2(Vh + (size_t)(r0 + u * NW) * D);
-#pragma unroll
-      for (int u = 0; u < 4; ++u) { acc[0] += v[u].x; acc[1] += v[u].y; }
+    for (int u = 0; u < 8; ++u) {
+      const bool in = r0 + u * NW < end;
+      if constexpr (PER == 4) {
+        const float4 v = in ? ld4(Vh + (size_t)(r0 + u * NW) * D) : make_float4(0.f, 0.f, 0.f, 0.f);
+        x[u][0] = v.x; x[u][1] = v.y; x[u][2] = v.z; x[u][3] = v.w;
+      } else {
+        const float2 v = in ? ld2(Vh + (size_t)(r0 + u * NW) * D) : make_float2(0.f, 0.f);
+        x[u][0] = v.x; x[u][1] = v.y;
+      }
     }
-  }
-  for (int r = r0; r < end; r += NW) {
-    if constexpr (PER == 4) {
-      float4 v = ld4(Vh + (size_t)r * D);
-      acc[0] += v.x; acc[1] += v.y; acc[2] += v.z; acc[3] += v.w;
-    } else {
-      float2 v = ld2(Vh + (size_t)r * D);
-      acc[0] += v.x; acc[1] += v.y;
-    }
+#pragma unroll
+    for (int t = 0; t < PER; ++t)
+      acc[t] += (double)(((x[0][t] + x[1][t]) + (x[2][t] + x[3][t])) + ((x[4][t] + x[5][t]) + (x[6][t] + x[7][t])));
   }
 #pragma unroll
   for (int t = 0; t < PER; ++t) red[w][lane * PER + t] = acc[t];
@@ -84,34 +78,50 @@ __global__ void __launch_bounds__(256) k_value_stats(const T* __restrict__ Vp, c
 #pragma unroll
   for (int t = 0; t < PER; ++t) mv[t] = vb[lane * PER + t];
   const size_t plane = (size_t)H * N;
-  for (int r = beg + w; r < end; r += NW) {
-    float v[PER];
-    if constexpr (PER == 4) {
-      float4 q = ld4(Vh + (size_t)r * D);
-      v[0] = q.x; v[1] = q.y; v[2] = q.z; v[3] = q.w;
-    } else {
-      float2 q = ld2(Vh + (size_t)r * D);
-      v[0] = q.x; v[1] = q.y;
-    }
-    float s1 = 0.f, s2 = 0.f, s3 = 0.f;
+  // per-key scalars, four rows per warp in flight with independent reductions
+  constexpr int RB = 4;
+  for (int r0 = beg + w; r0 < end; r0 += RB * NW) {
+    float s1[RB], s2[RB], s3[RB];
 #pragma unroll
-    for (int t = 0; t < PER; ++t) {
-      const float dv = mv[t] - v[t];
-      s1 = fmaf(dv, dv, s1);
-      s2 = fmaf(dv, v[t], s2);
-      s3 = fmaf(v[t], v[t], s3);
+    for (int u = 0; u < RB; ++u) {
+      const int r = r0 + u * NW;
+      float v[PER];
+      if constexpr (PER == 4) {
+        const float4 q = r < end ? ld4(Vh + (size_t)r * D) : make_float4(0.f, 0.f, 0.f, 0.f);
+        v[0] = q.x; v[1] = q.y; v[2] = q.z; v[3] = q.w;
+      } else {
+        const float2 q = r < end ? ld2(Vh + (size_t)r * D) : make_float2(0.f, 0.f);
+        v[0] = q.x; v[1] = q.y;
+      }
+      s1[u] = 0.f; s2[u] = 0.f; s3[u] = 0.f;
+#pragma unroll
+      for (int t = 0; t < PER; ++t) {
+        const float dv = mv[t] - v[t];
+        s1[u] = fmaf(dv, dv, s1[u]);
+        s2[u] = fmaf(dv, v[t], s2[u]);
+        s3[u] = fmaf(v[t], v[t], s3[u]);
+      }
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) {
-      s1 += __shfl_xor_sync(0xffffffffu, s1, o);
-      s2 += __shfl_xor_sync(0xffffffffu, s2, o);
-      s3 += __shfl_xor_sync(0xffffffffu, s3, o);
+#pragma unroll
+      for (int u = 0; u < RB; ++u) {
+        s1[u] += __shfl_xor_sync(0xffffffffu, s1[u], o);
+        s2[u] += __shfl_xor_sync(0xffffffffu, s2[u], o);
+        s3[u] += __shfl_xor_sync(0xffffffffu, s3[u], o);
+      }
     }
     if (lane == 0) {
-      const size_t i = (size_t)h * N + r;
-      ks[i] = s1;
-      ks[plane + i] = s2;
-      ks[2 * plane + i] = s3;
+#pragma unroll
+      for (int u = 0; u < RB; ++u) {
+        const int r = r0 + u * NW;
+        if (r < end) {
+          const size_t i = (size_t)h * N + r;
+          ks[i] = s1[u];
+          ks[plane + i] = s2[u];
+          ks[2 * plane + i] = s3[u];
+        }
+      }
     }
   }
 }
