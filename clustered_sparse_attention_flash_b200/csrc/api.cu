@@ -297,7 +297,7 @@ int svgear_forward(const void* Q, const void* K, const void* V, const svgear_par
   const int H = p->H, Nq = p->Nq, Nk = p->Nk, d = p->d, Cq = p->Cq, Ck = p->Ck, dt = p->dtype;
   const float sc = eff_scale(p);
   cudaStream_t st = S(stream);
-  cudaEvent_t ev[7] = {};
+  cudaEvent_t ev[9] = {};  // stage boundaries 0..6, then the attention kernel alone
   if (stats) {
     for (auto& e : ev)
       if (cudaEventCreate(&e) != cudaSuccess) return SVGEAR_ERR_CUDA;
@@ -325,9 +325,12 @@ int svgear_forward(const void* Q, const void* K, const void* V, const svgear_par
     e = route_run(L.E, L.counts_k, L.counts_q, H, Nk, Cq, Ck, p->rho, L.mask, L.sel, L.n_sel,
                   L.exec_pairs, st, p->budget == SVGEAR_BUDGET_GLOBAL ? L.M : nullptr, Nq);
   mark(5);
+  if (stats) attn_tc_time_next_kernel(ev[7], ev[8]);
   if (e == cudaSuccess)
     e = attn_run(L.Qp, L.Kp, L.Vp, L.off_q, L.off_k, L.perm_q, L.cent_k, L.vbar, L.sel, L.n_sel, dt,
                  H, Nq, Nk, d, Cq, Ck, sc, O, L.scratch, st);
+  const bool kernel_timed = stats && attn_tc_kernel_was_timed();
+  if (stats) attn_tc_time_next_kernel(nullptr, nullptr);
   mark(6);
   if (stats && e == cudaSuccess) {
     e = cudaStreamSynchronize(st);
@@ -337,6 +340,8 @@ int svgear_forward(const void* Q, const void* K, const void* V, const svgear_par
       stats->ms_kmeans_q = t[0]; stats->ms_kmeans_k = t[1]; stats->ms_permute = t[2];
       stats->ms_block_error = t[3]; stats->ms_route = t[4]; stats->ms_attn = t[5];
       cudaEventElapsedTime(&stats->ms_total, ev[0], ev[6]);
+      stats->ms_attn_kernel = stats->ms_attn;
+      if (kernel_timed) cudaEventElapsedTime(&stats->ms_attn_kernel, ev[7], ev[8]);
       std::vector<int64_t> ep(H);
       std::vector<int32_t> cq((size_t)H * Cq), ck((size_t)H * Ck), ns((size_t)H * Cq);
       e = cudaMemcpy(ep.data(), L.exec_pairs, H * sizeof(int64_t), cudaMemcpyDeviceToHost);

@@ -856,6 +856,11 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 int round_stage(int x) { return (x + BN - 1) / BN * BN; }
 
+// Events the next launch records around the attention kernel alone (set by
+// the forward when the caller asked for stage timings; per host thread).
+thread_local cudaEvent_t t_kernel_ev[2] = {nullptr, nullptr};
+thread_local bool t_kernel_ev_used = false;
+
 struct AttnWs {
   uint8_t *kh, *kl, *vh, *vl, *kpk, *vpk;
   int32_t* poff;
@@ -910,15 +915,30 @@ cudaError_t launch(const void* Qp, const void* Kp, const void* Vp, const int32_t
   e = cudaFuncGetAttributes(&fa, k_attn_tc<D>);
   if (e != cudaSuccess) return e;
   if ((long long)fa.numRegs * kThreads < 4LL * 32 * kRegsLow + 8LL * 32 * kRegsHigh) return cudaErrorInvalidValue;
+  const bool timed = t_kernel_ev[0] != nullptr;
+  if (timed) cudaEventRecord(t_kernel_ev[0], st);
   k_attn_tc<D><<<dim3(tmax, H), kThreads, smem, st>>>(
       static_cast<const bf16*>(Qp), w.kpk, w.vpk, w.npad, q_off, k_off, w.poff, perm_q, w.kh, w.kl, w.vh, w.vl,
       w.lc2, sel, n_sel, w.tiles, w.ntiles, tmax, Nq, Nk, Cq, Ck, Ckpad, scale * kLog2e,
       static_cast<bf16*>(O), status_word());
   note_launch();
+  if (timed) {
+    cudaEventRecord(t_kernel_ev[1], st);
+    t_kernel_ev[0] = t_kernel_ev[1] = nullptr;
+    t_kernel_ev_used = true;
+  }
   return cudaGetLastError();
 }
 
 }  // namespace
+
+void attn_tc_time_next_kernel(cudaEvent_t begin, cudaEvent_t end) {
+  t_kernel_ev[0] = begin;
+  t_kernel_ev[1] = end;
+  t_kernel_ev_used = false;
+}
+
+bool attn_tc_kernel_was_timed() { return t_kernel_ev_used; }
 
 bool attn_tc_supported(int d, int Ck) { return (d == 64 || d == 128) && Ck <= kMaxCkBits; }
 

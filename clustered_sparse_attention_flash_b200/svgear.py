@@ -50,7 +50,7 @@ class svgear_stats(ctypes.Structure):
                 ("ms_permute", ctypes.c_float), ("ms_block_error", ctypes.c_float),
                 ("ms_route", ctypes.c_float), ("ms_attn", ctypes.c_float),
                 ("ms_total", ctypes.c_float), ("exec_pairs", ctypes.c_int64),
-                ("comp_pairs", ctypes.c_int64)]
+                ("comp_pairs", ctypes.c_int64), ("ms_attn_kernel", ctypes.c_float)]
 
     def as_dict(self) -> Dict[str, float]:
         return {k: getattr(self, k) for k, _ in self._fields_}

@@ -115,6 +115,8 @@ typedef struct {
   float ms_total;
   int64_t exec_pairs;   /* sum over heads of sum_a |q_a| * sum_{c routed} |k_c| */
   int64_t comp_pairs;   /* sum over heads of sum_a |q_a| * #compensated non-empty c */
+  float ms_attn_kernel; /* the hybrid-attention kernel alone (ms_attn less its staging
+                           kernels); equal to ms_attn on the float32 path */
 } svgear_stats;
 
 /* Device pointers to the intermediates svgear_forward leaves in its workspace. */
