@@ -75,7 +75,7 @@ float eff_scale(const svgear_params* p) {
 struct FwdLayout {
   float *cent_q, *cent_k, *vbar, *key_scalars, *E, *M;
   int32_t *labels_q, *labels_k, *counts_q, *counts_k, *perm_q, *perm_k, *off_q, *off_k, *sel, *n_sel;
-  void *Qp, *Kp, *Vp, *scratch;
+  void *Qp, *Kp, *Vp, *scratch, *scratch_q;
   uint8_t* mask;
   int64_t* exec_pairs;
   size_t scratch_bytes, total;
@@ -107,14 +107,47 @@ FwdLayout layout(const svgear_params* p, void* ws) {
   L.sel = cv.take<int32_t>((size_t)H * Cq * Ck);
   L.n_sel = cv.take<int32_t>((size_t)H * Cq);
   L.exec_pairs = cv.take<int64_t>(H);
-  size_t sb = kmeans_ws_bytes(H, Nq, d, Cq);
-  sb = std::max(sb, kmeans_ws_bytes(H, Nk, d, Ck));
+  // The query clustering runs beside the key clustering, so it has scratch of its own.
+  L.scratch_q = cv.take<char>(kmeans_ws_bytes(H, Nq, d, Cq));
+  size_t sb = kmeans_ws_bytes(H, Nk, d, Ck);
   sb = std::max(sb, block_error_ws_bytes(H, Cq, Ck, d, p->dtype));
   sb = std::max(sb, attn_ws_bytes(H, Nq, Nk, d, Cq, Ck));
   L.scratch = cv.take<char>(sb);
   L.scratch_bytes = sb;
   L.total = cv.used();
   return L;
+}
+
+// A second stream per host thread and device, at the device's highest priority:
+// the key clustering and everything that follows it up to the block error run
+// there, the query clustering stays on the caller's stream and fills the SMs the
+// key chain leaves idle.  Fork and join are event waits, so the pair also records
+// into a CUDA graph captured on the caller's stream.
+struct SideStream {
+  cudaStream_t s = nullptr;
+  cudaEvent_t fork = nullptr, join = nullptr;
+};
+
+SideStream* side_stream() {
+  thread_local SideStream cache[64];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+  SideStream& c = cache[dev];
+  if (!c.s) {
+    int least = 0, greatest = 0;
+    if (cudaDeviceGetStreamPriorityRange(&least, &greatest) != cudaSuccess) return nullptr;
+    if (cudaStreamCreateWithPriority(&c.s, cudaStreamNonBlocking, greatest) != cudaSuccess) {
+      c.s = nullptr;
+      return nullptr;
+    }
+    if (cudaEventCreateWithFlags(&c.fork, cudaEventDisableTiming) != cudaSuccess ||
+        cudaEventCreateWithFlags(&c.join, cudaEventDisableTiming) != cudaSuccess) {
+      cudaStreamDestroy(c.s);
+      c = SideStream{};
+      return nullptr;
+    }
+  }
+  return &c;
 }
 
 }  // namespace
@@ -297,6 +330,8 @@ int svgear_forward(const void* Q, const void* K, const void* V, const svgear_par
   const int H = p->H, Nq = p->Nq, Nk = p->Nk, d = p->d, Cq = p->Cq, Ck = p->Ck, dt = p->dtype;
   const float sc = eff_scale(p);
   cudaStream_t st = S(stream);
+  SideStream* side = side_stream();
+  if (!side) return SVGEAR_ERR_CUDA;
   cudaEvent_t ev[9] = {};  // stage boundaries 0..6, then the attention kernel alone
   if (stats) {
     for (auto& e : ev)
@@ -305,17 +340,33 @@ int svgear_forward(const void* Q, const void* K, const void* V, const svgear_par
   auto mark = [&](int i) { if (stats) cudaEventRecord(ev[i], st); };
   cudaError_t e = cudaSuccess;
   mark(0);
-  e = kmeans_run(Q, dt, H, Nq, d, Cq, p->iters, init_q, L.cent_q, L.labels_q, L.counts_q, L.off_q,
-                 L.perm_q, L.scratch, st);
-  mark(1);
+  // The key chain on the side stream, the query clustering and gather on `st`.
+  e = cudaEventRecord(side->fork, st);
+  if (e == cudaSuccess) e = cudaStreamWaitEvent(side->s, side->fork, 0);
+  const bool forked = e == cudaSuccess;
+  cudaError_t ek = e, ej = e;
+  if (forked) {
+    cudaStream_t sk = side->s;
+    ek = kmeans_run(K, dt, H, Nk, d, Ck, p->iters, init_k, L.cent_k, L.labels_k, L.counts_k,
+                    L.off_k, L.perm_k, L.scratch, sk);
+    if (stats) cudaEventRecord(ev[2], sk);
+    if (ek == cudaSuccess) ek = gather_rows(K, dt, L.perm_k, H, Nk, d, L.Kp, sk);
+    if (ek == cudaSuccess) ek = gather_rows(V, dt, L.perm_k, H, Nk, d, L.Vp, sk);
+    if (ek == cudaSuccess) ek = value_stats(L.Vp, dt, L.off_k, H, Nk, d, Ck, L.vbar, L.key_scalars, sk);
+    // Recorded whatever happened above: `st` always waits for the side stream.
+    ej = cudaEventRecord(side->join, sk);
+  }
   if (e == cudaSuccess)
-    e = kmeans_run(K, dt, H, Nk, d, Ck, p->iters, init_k, L.cent_k, L.labels_k, L.counts_k, L.off_k,
-                   L.perm_k, L.scratch, st);
-  mark(2);
+    e = kmeans_run(Q, dt, H, Nq, d, Cq, p->iters, init_q, L.cent_q, L.labels_q, L.counts_q,
+                   L.off_q, L.perm_q, L.scratch_q, st);
+  mark(1);
   if (e == cudaSuccess) e = gather_rows(Q, dt, L.perm_q, H, Nq, d, L.Qp, st);
-  if (e == cudaSuccess) e = gather_rows(K, dt, L.perm_k, H, Nk, d, L.Kp, st);
-  if (e == cudaSuccess) e = gather_rows(V, dt, L.perm_k, H, Nk, d, L.Vp, st);
-  if (e == cudaSuccess) e = value_stats(L.Vp, dt, L.off_k, H, Nk, d, Ck, L.vbar, L.key_scalars, st);
+  if (forked) {
+    if (ej == cudaSuccess) ej = cudaStreamWaitEvent(st, side->join, 0);
+    if (ej != cudaSuccess) cudaStreamSynchronize(side->s);
+  }
+  if (e == cudaSuccess) e = ek;
+  if (e == cudaSuccess) e = ej;
   mark(3);
   if (e == cudaSuccess)
     e = block_error_run(L.cent_q, L.cent_k, L.vbar, L.Kp, L.Vp, L.off_k, L.key_scalars, dt, H, Nk, d,
@@ -336,6 +387,9 @@ int svgear_forward(const void* Q, const void* K, const void* V, const svgear_par
     e = cudaStreamSynchronize(st);
     float t[6] = {};
     for (int i = 0; i < 6 && e == cudaSuccess; ++i) e = cudaEventElapsedTime(&t[i], ev[i], ev[i + 1]);
+    // Both clusterings start at ev[0]: ev[1] ends the query one, ev[2] (on the
+    // side stream) the key one; the permute stage runs from ev[2] to the join.
+    if (e == cudaSuccess) e = cudaEventElapsedTime(&t[1], ev[0], ev[2]);
     if (e == cudaSuccess) {
       stats->ms_kmeans_q = t[0]; stats->ms_kmeans_k = t[1]; stats->ms_permute = t[2];
       stats->ms_block_error = t[3]; stats->ms_route = t[4]; stats->ms_attn = t[5];

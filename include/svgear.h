@@ -109,7 +109,10 @@ typedef struct {
                    read by svgear_forward only */
 } svgear_params;
 
-/* Per-stage device times of one svgear_forward call (CUDA events). */
+/* Per-stage device times of one svgear_forward call (CUDA events).  The two
+ * clusterings run side by side, so ms_kmeans_q and ms_kmeans_k both start at the
+ * call's start and overlap; ms_permute runs from the end of the key clustering
+ * to the point where both permuted halves are ready. */
 typedef struct {
   float ms_kmeans_q, ms_kmeans_k, ms_permute, ms_block_error, ms_route, ms_attn;
   float ms_total;
@@ -304,6 +307,13 @@ SVGEAR_API int svgear_hybrid_attn(const void* Qp, const void* Kp, const void* Vp
 /* ---------------------------------------------------------------------------
  * The whole operator: (1) -> (1') -> (2) -> (3) -> (4) on one stream
  * ((3') instead of (3) when p->budget is SVGEAR_BUDGET_GLOBAL).
+ *   The key clustering, the key/value gathers and (1') run on a second,
+ *   highest-priority stream the library keeps per host thread and device,
+ *   forked from `stream` by an event and joined back before (2), while the
+ *   query clustering runs on `stream` beside them; to the caller the call still
+ *   behaves as work on `stream` alone (ordering, graph capture).  Concurrent
+ *   calls from one host thread on different streams share that second stream
+ *   and serialise their key chains.
  *   Q [H,Nq,d], K/V [H,Nk,d], O [H,Nq,d] in `dtype`.
  *   init_q [H,Cq,d] / init_k [H,Ck,d] float32 k-means initial centroids
  *   (NULL: deterministic init, see svgear_kmeans).
