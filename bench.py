@@ -149,13 +149,12 @@ def _peaks():
 
 # DRAM traffic of the attention kernel from one ncu capture (dram__bytes_read.sum
 # + dram__bytes_write.sum of k_attn_tc on the first 4 heads of the Wan-shaped
-# workload: 278.7 + 67.0 = 345.7 MB, i.e. 86.4 MB per head; traffic grows with
+# workload: 282.3 + 65.9 = 348.3 MB, i.e. 87.1 MB per head; traffic grows with
 # the heads).  The figure holds only for the kernel sources it was taken on,
-# identified by hash (the hash was moved once, over a change to the host-side
-# launch code only: the kernel body is the captured one).
-_ATTN_TRAFFIC = {"bytes_per_head": 345.679e6 / 4, "workload": "wan",
+# identified by hash.
+_ATTN_TRAFFIC = {"bytes_per_head": 348.272e6 / 4, "workload": "wan",
                  "sources": ("attn_tc.cu", "attn_tc.cuh", "tc_common.cuh"),
-                 "sha1": "14a456b5f52dc2e79000ef0f5e17cbd02c80e611"}
+                 "sha1": "25131a08ccbecf1c68f900f56a846013d0e37f89"}
 
 
 def attn_traffic(cfg):

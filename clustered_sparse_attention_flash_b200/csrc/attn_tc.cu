@@ -710,6 +710,54 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc::tmem_ld32(tmem + lane_base + scol + 64u, *reinterpret_cast<uint32_t(*)[32]>(v + 64));
       tc::tmem_ld32(tmem + lane_base + scol + 96u, *reinterpret_cast<uint32_t(*)[32]>(v + 96));
       tc::tmem_ld_wait();
+      // Routed stage of rows whose running maximum is already a non-negative
+      // real logit: the exponentials are taken against it straight away (the
+      // padding keys' share 2^(0 - m) <= 1 comes off the row sum, as on the
+      // fast path below) while the stage's maximum is found in the same pass.
+      // P stays in registers until that maximum is known, so S[t] is still
+      // intact when a row's maximum grew by more than 2^8 (rare once a row has
+      // seen a few stages): then S is reloaded and the stage takes the path
+      // below, on the raw formula (every reference maximum is >= 0) and
+      // without touching the released bias slot again.
+      bool spec_failed = false;
+      int npad_spec = 0;
+      if (j < n_ex && __all_sync(0xffffffffu, m_used >= 0.f)) {
+        npad_spec = BN - nv_s[sb];
+        const uint64_t negm = f2(-m_used, -m_used);
+        const uint64_t sc2 = f2(scale2, scale2);
+        uint32_t pk[64];
+        uint64_t r2[2] = {0ull, 0ull};
+        float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+        for (int i = 0; i < 64; ++i) {
+          const uint64_t x = f2_fma(f2(__uint_as_float(v[2 * i]), __uint_as_float(v[2 * i + 1])), sc2, negm);
+          const float p0 = ex2(f2_lo(x)), p1 = ex2(f2_hi(x));
+          r2[i & 1] = f2_add(r2[i & 1], f2(p0, p1));
+          pk[i] = pack_bf16(p0, p1);
+          m4[i & 3] = tc::fmax3(m4[i & 3], __uint_as_float(v[2 * i]), __uint_as_float(v[2 * i + 1]));
+        }
+        __syncwarp();
+        if (lane == 0) tc::mbar_arrive(b_empty + sb);
+        const float mxs = fmaxf(tc::fmax3(m4[0], m4[1], m4[2]), m4[3]) * scale2;
+        if (!__any_sync(0xffffffffu, mxs > m_used + 8.f)) {
+#pragma unroll
+          for (int q = 0; q < 4; ++q)
+            tc::tmem_st16(tmem + lane_base + scol + (uint32_t)(q * 16),
+                          *reinterpret_cast<const uint32_t(*)[16]>(pk + 16 * q));
+          tc::tmem_st_wait();
+          const uint64_t r = f2_add(r2[0], r2[1]);
+          l += (f2_lo(r) + f2_hi(r)) - (float)npad_spec * ex2(-m_used);
+          tc::tc_fence_before();
+          tc::mbar_arrive(p_full + t);
+          continue;
+        }
+        spec_failed = true;
+        tc::tmem_ld32(tmem + lane_base + scol, *reinterpret_cast<uint32_t(*)[32]>(v));
+        tc::tmem_ld32(tmem + lane_base + scol + 32u, *reinterpret_cast<uint32_t(*)[32]>(v + 32));
+        tc::tmem_ld32(tmem + lane_base + scol + 64u, *reinterpret_cast<uint32_t(*)[32]>(v + 64));
+        tc::tmem_ld32(tmem + lane_base + scol + 96u, *reinterpret_cast<uint32_t(*)[32]>(v + 96));
+        tc::tmem_ld_wait();
+      }
       // Routed stage, fast path: padding and tail keys have zero key rows, so
       // their logits are exactly 0 and their value rows are 0.  When the raw
       // maximum of the stage is positive it is a real key's, the scale and
@@ -730,7 +778,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int k = 0; k < 8; ++k)
               m8[k] = tc::fmax3(m8[k], __uint_as_float(v[i + 2 * k]), __uint_as_float(v[i + 2 * k + 1]));
           const float mr = fmaxf(tc::fmax3(m8[0], m8[1], m8[2]), tc::fmax3(tc::fmax3(m8[3], m8[4], m8[5]), m8[6], m8[7]));
-          raw = __all_sync(0xffffffffu, mr > 0.f);
+          raw = spec_failed || __all_sync(0xffffffffu, mr > 0.f);
           mx = mr * scale2;
         }
         if (!raw) {
@@ -757,10 +805,11 @@ __global__ void __launch_bounds__(kThreads, 1)
           mx = fmaxf(tc::fmax3(m8[0], m8[1], m8[2]), tc::fmax3(tc::fmax3(m8[3], m8[4], m8[5]), m8[6], m8[7]));
         }
       }
-      const int npad = raw ? BN - nv_s[sb] : 0;
-      // the bias is read: release the stage's bias slot(s) on this warp's behalf
+      const int npad = spec_failed ? npad_spec : raw ? BN - nv_s[sb] : 0;
+      // the bias is read: release the stage's bias slot(s) on this warp's
+      // behalf (a failed speculative stage released its slot already)
       __syncwarp();
-      if (lane == 0)
+      if (lane == 0 && !spec_failed)
         for (int q = 0; q < nparts(j); ++q) tc::mbar_arrive(b_empty + (u0 + q) % kBSlots);
       // lazy rescale: a row whose maximum grew by more than 2^8 rescales O[t]
       // and l.  The tensor-memory accesses are warp-collective, so the warp
