@@ -149,12 +149,12 @@ def _peaks():
 
 # DRAM traffic of the attention kernel from one ncu capture (dram__bytes_read.sum
 # + dram__bytes_write.sum of k_attn_tc on the first 4 heads of the Wan-shaped
-# workload: 282.3 + 65.9 = 348.3 MB, i.e. 87.1 MB per head; traffic grows with
+# workload: 278.3 + 63.5 = 341.9 MB, i.e. 85.5 MB per head; traffic grows with
 # the heads).  The figure holds only for the kernel sources it was taken on,
 # identified by hash.
-_ATTN_TRAFFIC = {"bytes_per_head": 348.272e6 / 4, "workload": "wan",
+_ATTN_TRAFFIC = {"bytes_per_head": 341.860e6 / 4, "workload": "wan",
                  "sources": ("attn_tc.cu", "attn_tc.cuh", "tc_common.cuh"),
-                 "sha1": "25131a08ccbecf1c68f900f56a846013d0e37f89"}
+                 "sha1": "f6d5338f36b9197d3fb37e0b59c2045f09d1d62d"}
 
 
 def attn_traffic(cfg):

@@ -713,12 +713,16 @@ __global__ void __launch_bounds__(kThreads, 1)
       // Routed stage of rows whose running maximum is already a non-negative
       // real logit: the exponentials are taken against it straight away (the
       // padding keys' share 2^(0 - m) <= 1 comes off the row sum, as on the
-      // fast path below) while the stage's maximum is found in the same pass.
-      // P stays in registers until that maximum is known, so S[t] is still
-      // intact when a row's maximum grew by more than 2^8 (rare once a row has
-      // seen a few stages): then S is reloaded and the stage takes the path
-      // below, on the raw formula (every reference maximum is >= 0) and
-      // without touching the released bias slot again.
+      // fast path below), without a maximum pass.  The stage is accepted when
+      // every row's sum of the 128 terms is at most 2^16: then no term exceeds
+      // 2^16, which bf16 P and the float32 accumulators carry without loss
+      // (the reference maximum only has to keep the terms finite; the result
+      // does not depend on it).  P stays in registers until then, so S[t] is
+      // still intact when a row's sum is larger (its maximum grew by more than
+      // 2^9 at least, rare once a row has seen a few stages): S is reloaded and
+      // the stage takes the path below, which finds the maximum and rescales,
+      // on the raw formula (every reference maximum is >= 0) and without
+      // touching the released bias slot again.
       bool spec_failed = false;
       int npad_spec = 0;
       if (j < n_ex && __all_sync(0xffffffffu, m_used >= 0.f)) {
@@ -727,26 +731,24 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint64_t sc2 = f2(scale2, scale2);
         uint32_t pk[64];
         uint64_t r2[2] = {0ull, 0ull};
-        float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
         for (int i = 0; i < 64; ++i) {
           const uint64_t x = f2_fma(f2(__uint_as_float(v[2 * i]), __uint_as_float(v[2 * i + 1])), sc2, negm);
           const float p0 = ex2(f2_lo(x)), p1 = ex2(f2_hi(x));
           r2[i & 1] = f2_add(r2[i & 1], f2(p0, p1));
           pk[i] = pack_bf16(p0, p1);
-          m4[i & 3] = tc::fmax3(m4[i & 3], __uint_as_float(v[2 * i]), __uint_as_float(v[2 * i + 1]));
         }
         __syncwarp();
         if (lane == 0) tc::mbar_arrive(b_empty + sb);
-        const float mxs = fmaxf(tc::fmax3(m4[0], m4[1], m4[2]), m4[3]) * scale2;
-        if (!__any_sync(0xffffffffu, mxs > m_used + 8.f)) {
+        const uint64_t rs = f2_add(r2[0], r2[1]);
+        const float tot = f2_lo(rs) + f2_hi(rs);
+        if (__all_sync(0xffffffffu, tot <= 65536.f)) {
 #pragma unroll
           for (int q = 0; q < 4; ++q)
             tc::tmem_st16(tmem + lane_base + scol + (uint32_t)(q * 16),
                           *reinterpret_cast<const uint32_t(*)[16]>(pk + 16 * q));
           tc::tmem_st_wait();
-          const uint64_t r = f2_add(r2[0], r2[1]);
-          l += (f2_lo(r) + f2_hi(r)) - (float)npad_spec * ex2(-m_used);
+          l += tot - (float)npad_spec * ex2(-m_used);
           tc::tc_fence_before();
           tc::mbar_arrive(p_full + t);
           continue;

@@ -26,7 +26,7 @@ def test_attention_traffic_only_for_its_capture():
     t = bench.attn_traffic(wan)
     if _sources_hash() == bench._ATTN_TRAFFIC["sha1"]:
         assert t == pytest.approx(bench._ATTN_TRAFFIC["bytes_per_head"] * wan.H)
-        assert bench.attn_traffic(wan.with_(H=4)) == pytest.approx(348.272e6)
+        assert bench.attn_traffic(wan.with_(H=4)) == pytest.approx(341.860e6)
     else:
         assert t is None
 
