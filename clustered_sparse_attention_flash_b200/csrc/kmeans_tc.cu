@@ -8,13 +8,16 @@
 // tensor memory, 128 centroid columns per accumulator slot).  The epilogue
 // subtracts ||mu_c||^2 / 2, writes the column index into the low mantissa bits
 // of the score (so one float carries score and index, and no two columns tie)
-// and keeps the three largest packed scores b1 >= b2 >= b3 per token.
+// and keeps, per token, the two largest packed scores b1 >= b2 exactly and an
+// upper bound b2 >= b3 of the third largest.
 //
 // Every packed score is within E of the exact s_c (bf16 rounding of mu, the
 // fp32 accumulation inside the MMA, the subtraction, the index bits; bound
 // below), so the exact best column has a packed score >= b1 - 2E:
 //   b2 <  b1 - 2E            -> the label is the column of b1 (exact);
-//   b3 <  b1 - 2E <= b2      -> one of the columns of b1, b2: decided in float64;
+//   b3 <  b1 - 2E <= b2      -> one of the columns of b1, b2: decided in float64
+//                               (b3 bounds the third score from above, so no
+//                               third column is within the bound);
 //   otherwise                -> every centroid is checked in float64.
 // Ties in float64 go to the smaller index, so labels equal the exact argmin.
 //
@@ -379,9 +382,13 @@ __device__ __forceinline__ float score_error(float xn, const Bounds& b, float id
 
 // Insert two packed scores into the running top three (b1 >= b2 >= b3): the
 // k-th largest of two sorted lists is the largest min(A_i, B_j) over i + j = k.
+// b1 and b2 stay exact.  For the third, lo stands in for min(b1, lo): equal
+// unless both new scores exceed b1, and never smaller, so b3 stays an upper
+// bound of the third largest (and at most b2), which is all the decision and
+// the merges need; it saves one instruction per pair of columns.
 __device__ __forceinline__ void top3_add2(float& b1, float& b2, float& b3, float p0, float p1) {
   const float hi = fmaxf(p0, p1), lo = fminf(p0, p1);
-  const float n3 = tc::fmax3(b3, fminf(b2, hi), fminf(b1, lo));
+  const float n3 = tc::fmax3(b3, fminf(b2, hi), lo);
   const float n2 = tc::fmax3(b2, fminf(b1, hi), lo);
   b1 = fmaxf(b1, hi);
   b2 = n2;
