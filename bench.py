@@ -24,7 +24,6 @@ import os
 import statistics
 import subprocess
 import sys
-import tempfile
 import time
 
 ROOT = os.path.dirname(os.path.abspath(__file__))
@@ -87,41 +86,68 @@ def generate(cfg):
 
 
 class Clocks:
-    """nvidia-smi sampling of SM clocks and throttle reasons over a region."""
+    """nvidia-smi sampling of SM clocks and throttle reasons over a region.
+
+    A reader thread stamps every sample with the host clock.  Entering waits
+    (at most a few seconds) for the first sample, so that the sampler is up
+    before the region starts; the summary keeps the samples taken inside the
+    region plus the first one after it (a region shorter than the sampling
+    interval still gets one)."""
     FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    INTERVAL_MS = 50
 
     def __init__(self, gpu_id):
         self.gpu_id = gpu_id
         self.proc = None
-        self.path = None
+        self.lines = []          # (host time, line)
+        self.t0 = self.t1 = None
+        self.thread = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append((time.monotonic(), line))
 
     def __enter__(self):
+        import threading
         try:
-            fd, self.path = tempfile.mkstemp(suffix=".csv")
-            os.close(fd)
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", str(self.gpu_id), f"--query-gpu={self.FIELDS}",
-                 "--format=csv,noheader,nounits", "-lms", "200", "-f", self.path],
-                stdout=subprocess.DEVNULL, stderr=subprocess.DEVNULL)
+                 "--format=csv,noheader,nounits", "-lms", str(self.INTERVAL_MS)],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+            deadline = time.monotonic() + 5.0
+            while not self.lines and time.monotonic() < deadline and self.proc.poll() is None:
+                time.sleep(0.01)
         except Exception:
             self.proc = None
+        self.t0 = time.monotonic()
         return self
 
     def __exit__(self, *a):
+        self.t1 = time.monotonic()
         if self.proc is not None:
+            deadline = self.t1 + 3.0 * self.INTERVAL_MS / 1e3 + 0.5
+            while not any(t > self.t1 for t, _ in self.lines) and time.monotonic() < deadline \
+                    and self.proc.poll() is None:
+                time.sleep(0.01)
             self.proc.terminate()
             try:
                 self.proc.wait(timeout=5)
             except Exception:
                 self.proc.kill()
+            if self.thread is not None:
+                self.thread.join(timeout=2)
 
     def summary(self):
-        if not self.path or not os.path.exists(self.path):
+        if self.proc is None:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"]}
+        inside = [ln for t, ln in self.lines if self.t0 <= t <= self.t1]
+        after = [ln for t, ln in self.lines if t > self.t1][:1]
         rows = []
-        for line in open(self.path):
+        for line in inside + after:
             f = [x.strip() for x in line.split(",")]
             if len(f) < 8:
                 continue
@@ -129,7 +155,6 @@ class Clocks:
                 rows.append((float(f[0]), float(f[1]), f[4], f[5], f[6], f[7]))
             except ValueError:
                 continue
-        os.unlink(self.path)
         if not rows:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
         names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")

@@ -1,7 +1,7 @@
 """bench.py's host-side helpers, no GPU: the DRAM-traffic figure is reported
 only for the workload and kernel sources it was captured on, the stress
-sweep's trend test, the workload description and the generator's
-configuration override."""
+sweep's trend test, the workload description, the generator's configuration
+override and the clock sampler (against a stand-in nvidia-smi)."""
 import hashlib
 import os
 
@@ -55,3 +55,29 @@ def test_generator_honours_the_config_it_is_given():
     for x, y in zip(b, c):
         np.testing.assert_array_equal(x, y)
     assert a[3].shape == (base.Cq, base.d) and a[4].shape == (base.Ck, base.d)
+
+
+def test_clock_sampler_covers_a_short_region(tmp_path, monkeypatch):
+    # A stand-in nvidia-smi that starts slowly and then prints one CSV sample
+    # every 50 ms; a region much shorter than the start-up still gets samples
+    # and the throttle reasons are read from the right columns.
+    fake = tmp_path / "nvidia-smi"
+    fake.write_text("#!/bin/sh\nsleep 0.3\nwhile true; do\n"
+                    "  echo '1965, 1965, 700.5, 0x4, Not Active, Not Active, Not Active, Active'\n"
+                    "  sleep 0.05\ndone\n")
+    fake.chmod(0o755)
+    monkeypatch.setenv("PATH", f"{tmp_path}{os.pathsep}{os.environ.get('PATH', '')}")
+    import time
+    with bench.Clocks(0) as clk:
+        time.sleep(0.02)
+    out = clk.summary()
+    assert out["samples"] >= 1
+    assert out["sm_mhz"] == 1965.0 and out["sm_max_mhz"] == 1965.0
+    assert out["reasons"] == ["sw_power_cap"]
+
+
+def test_clock_sampler_without_nvidia_smi(tmp_path, monkeypatch):
+    monkeypatch.setenv("PATH", str(tmp_path))
+    with bench.Clocks(0) as clk:
+        pass
+    assert clk.summary()["reasons"] == ["unavailable"]
