@@ -389,11 +389,12 @@ def run_shard_heads(a, cfg, rho):
         torch.cuda.synchronize(dev)
         ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         l0 = sv.svgear_launch_count()
-        ev0.record(stream)
-        for _ in range(a.steps):
-            step()
-        ev1.record(stream)
-        torch.cuda.synchronize(dev)
+        with Clocks(local) as clk:
+            ev0.record(stream)
+            for _ in range(a.steps):
+                step()
+            ev1.record(stream)
+            torch.cuda.synchronize(dev)
         launches = sv.svgear_launch_count() - l0
         if dist is not None:
             dist.barrier()
@@ -406,7 +407,7 @@ def run_shard_heads(a, cfg, rho):
                     "config": {"workload": _workload(cfg, rho),
                                "parallelism": f"heads sharded x{world} ({e - b} heads on rank 0), "
                                               f"all-gather of O over the process group"},
-                    "gpu_launches": launches}
+                    "gpu_launches": launches, "clocks": clk.summary()}
             print(json.dumps(line), flush=True)
     finally:
         if dist is not None:
