@@ -298,24 +298,31 @@ __global__ void __launch_bounds__(kBeThreads, 1)
           if (cend == k1) flush();
           continue;
         }
-        // cluster boundaries inside the chunk: walk its keys; keys of other
-        // groups' clusters are passed over (every decision is block-uniform)
-        float part = 0.f;
-#pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          const int j = k0 + i;
-          if (j >= k1 || !(c < c_hi)) break;
-          if (j < cbeg) continue;          // another group's cluster
-          const float4 e = sc[q0 + i];
-          const float w = neg_expm1(__uint_as_float(v[i]) - Lc);
-          part += fmaxf(fmaf(w, fmaf(w, e.z, 2.f * e.y), e.x), 0.f);
-          if (j + 1 == cend) {             // the cluster ends here
-            acc += (double)part;
-            part = 0.f;
-            flush();
+        // cluster boundaries inside the chunk: one segment of the current
+        // cluster at a time (keys of other groups' clusters are passed over;
+        // every decision is block-uniform), its keys summed in order by a
+        // predicated pass over the chunk, so the flush is emitted once
+        int i0 = 0;
+        const int iend = k1 - k0;
+        while (i0 < iend && c < c_hi) {
+          if (k0 + i0 < cbeg) {            // another group's cluster
+            i0 = min(cbeg - k0, iend);
+            continue;
           }
+          const int i1 = min(cend - k0, iend);
+          float part = 0.f;
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            if (i >= i0 && i < i1) {
+              const float4 e = sc[q0 + i];
+              const float w = neg_expm1(__uint_as_float(v[i]) - Lc);
+              part += fmaxf(fmaf(w, fmaf(w, e.z, 2.f * e.y), e.x), 0.f);
+            }
+          }
+          acc += (double)part;
+          i0 = i1;
+          if (k0 + i1 == cend) flush();    // the cluster ends in this chunk
         }
-        acc += (double)part;
       }
       tc::tc_fence_before();
       __syncwarp();

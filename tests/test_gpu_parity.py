@@ -325,6 +325,41 @@ def test_forward_many_routed_clusters(N, Ck, rho):
     check_forward_given_gpu_clusters(views, host(O)[0], 0, q[0], k[0], v[0], Cq, Ck, rho, s, "bf16", rows=rows)
 
 
+def test_forward_row_maximum_grows_late():
+    """One key cluster whose logits exceed every other key's by about 20
+    (natural units) for every query: in the blocks whose stage order brings
+    it after the first stage, the running maximum of every row grows by far
+    more than 2^9 there, so the attention kernel's speculative pass rejects
+    that stage (row sums above 2^16), reloads S and rescales.  With rho = 1
+    every cluster is routed, so the output is dense attention."""
+    N, d, Cq, Ck = 8192, 128, 8, 64
+    q, k, v = _small(N, d, 41, "bf16")
+    rng = np.random.default_rng(42)
+    u = rng.standard_normal(d)
+    u /= np.linalg.norm(u)
+    hot = rng.choice(N, size=256, replace=False)
+    from clustered_sparse_attention_flash_b200.synth import to_bf16_f32
+    k = k.copy()
+    k[0, hot] += 15.0 * u
+    q = q + 15.0 * u
+    q, k = to_bf16_f32(q.astype(np.float32)), to_bf16_f32(k.astype(np.float32))
+    s = 1 / math.sqrt(d)
+    iq, ik = q[:, :Cq].copy(), k[:, :Ck].copy()
+    ik[0, 0] = k[0, hot[0]]                      # one initial centroid among the hot keys
+    bf = torch.bfloat16
+    O, ws, p, _ = sv.forward(dev(q, bf), dev(k, bf), dev(v, bf), Cq, Ck, 3, 1.0, s, dev(iq), dev(ik))
+    torch.cuda.synchronize()
+    assert sv.svgear_get_status() == sv.SVGEAR_OK
+    views = sv.view_tensors(p, ws)
+    lk = host(views["labels_k"])[0]
+    hot_clusters = set(lk[hot].tolist())
+    assert not (hot_clusters & set(np.delete(lk, hot).tolist())), "hot keys share a cluster with others"
+    assert (host(views["mask"])[0][:, host(views["counts_k"])[0] > 0] == 1).all()
+    rows = np.random.default_rng(3).choice(N, size=768, replace=False)
+    want = ora.dense_attention(q[0][rows], k[0], v[0], s)
+    assert_close(host(O)[0][rows], want, *OUT_TOL["bf16"], "late maximum growth")
+
+
 def test_forward_empty_key_cluster():
     """An initial centroid far from every key never gains members: the
     cluster stays empty, is never routed and contributes no compensation."""
