@@ -325,14 +325,16 @@ def test_forward_many_routed_clusters(N, Ck, rho):
     check_forward_given_gpu_clusters(views, host(O)[0], 0, q[0], k[0], v[0], Cq, Ck, rho, s, "bf16", rows=rows)
 
 
-def test_forward_row_maximum_grows_late():
+@pytest.mark.parametrize("d", [64, 128])
+def test_forward_row_maximum_grows_late(d):
     """One key cluster whose logits exceed every other key's by about 20
     (natural units) for every query: in the blocks whose stage order brings
     it after the first stage, the running maximum of every row grows by far
     more than 2^9 there, so the attention kernel's speculative pass rejects
     that stage (row sums above 2^16), reloads S and rescales.  With rho = 1
-    every cluster is routed, so the output is dense attention."""
-    N, d, Cq, Ck = 8192, 128, 8, 64
+    every cluster is routed, so the output is dense attention.  Both head
+    dimensions of the tensor-core kernel."""
+    N, Cq, Ck = 8192, 8, 64
     q, k, v = _small(N, d, 41, "bf16")
     rng = np.random.default_rng(42)
     u = rng.standard_normal(d)
