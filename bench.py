@@ -179,7 +179,7 @@ def _peaks():
 # identified by hash.
 _ATTN_TRAFFIC = {"bytes_per_head": 341.860e6 / 4, "workload": "wan",
                  "sources": ("attn_tc.cu", "attn_tc.cuh", "tc_common.cuh"),
-                 "sha1": "f6d5338f36b9197d3fb37e0b59c2045f09d1d62d"}
+                 "sha1": "bd86ed4d39fdb3b58578bccfa9fbbdd4d2887eb7"}
 
 
 def attn_traffic(cfg):

@@ -30,7 +30,8 @@
 // tiles halves the key / value traffic from L2 per FLOP, which is what bounds
 // a one-tile block.
 // Warp roles (12 warps):
-//   warp 0      tensor-memory allocation, MMA issue (one thread) in the order
+//   warp 0      tensor-memory allocation and the MMA issue loop (run by the
+//               whole warp, one elected lane issues) in the order
 //               P.V_0(j), S_0(j+1), P.V_1(j), S_1(j+1): while the tensor core
 //               works for one query tile the other tile's softmax runs;
 //   warps 1-3   load the two query tiles; warps 1 and 2 then produce the
@@ -40,8 +41,10 @@
 //               query row, all 128 keys of each stage): running maximum, row
 //               sum, lazy rescale of the tile's accumulator O[t] when the
 //               maximum grows by more than 2^8, P = 2^(x - m) in bf16 over the
-//               S columns of the tile; at the end O / l is stored through
-//               perm_q.
+//               S columns of the tile; most routed stages take a speculative
+//               pass against the running maximum with no maximum pass
+//               (accepted when no term can exceed 2^16); at the end O / l is
+//               stored through perm_q.
 // Tensor memory (512 columns): S[t] [128 t, 128 t + 128), O[t]
 // [256 + d t, 256 + d t + d); P[t] lives in the first 64 columns of S[t].
 // Every decision that guards a warp-collective tensor-memory access is made
@@ -86,16 +89,8 @@ __device__ __forceinline__ uint64_t f2(float lo, float hi) {
   asm("mov.b64 %0, {%1, %2};" : "=l"(d) : "f"(lo), "f"(hi));
   return d;
 }
-__device__ __forceinline__ float f2_lo(uint64_t x) {
-  float lo, hi;
-  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(x));
-  return lo;
-}
-__device__ __forceinline__ float f2_hi(uint64_t x) {
-  float lo, hi;
-  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(x));
-  return hi;
-}
+__device__ __forceinline__ float f2_lo(uint64_t x) { return __uint_as_float((uint32_t)x); }
+__device__ __forceinline__ float f2_hi(uint64_t x) { return __uint_as_float((uint32_t)(x >> 32)); }
 __device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
   uint64_t d;
   asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
