@@ -176,7 +176,8 @@ def _peaks():
 # + dram__bytes_write.sum of k_attn_tc on the first 4 heads of the Wan-shaped
 # workload: 278.3 + 63.5 = 341.9 MB, i.e. 85.5 MB per head; traffic grows with
 # the heads).  The figure holds only for the kernel sources it was taken on,
-# identified by hash.
+# identified by hash (moved only over changes that left the device code as
+# captured: comments and host-side code).
 _ATTN_TRAFFIC = {"bytes_per_head": 341.860e6 / 4, "workload": "wan",
                  "sources": ("attn_tc.cu", "attn_tc.cuh", "tc_common.cuh"),
                  "sha1": "bd86ed4d39fdb3b58578bccfa9fbbdd4d2887eb7"}
