@@ -313,7 +313,9 @@ SVGEAR_API int svgear_hybrid_attn(const void* Qp, const void* Kp, const void* Vp
  *   query clustering runs on `stream` beside them; to the caller the call still
  *   behaves as work on `stream` alone (ordering, graph capture).  Concurrent
  *   calls from one host thread on different streams share that second stream
- *   and serialise their key chains.
+ *   and serialise their key chains.  The first call on a host thread creates
+ *   that stream and sets the kernels' shared-memory attributes: make it outside
+ *   stream capture before recording svgear_forward into a CUDA graph.
  *   Q [H,Nq,d], K/V [H,Nk,d], O [H,Nq,d] in `dtype`.
  *   init_q [H,Cq,d] / init_k [H,Ck,d] float32 k-means initial centroids
  *   (NULL: deterministic init, see svgear_kmeans).
