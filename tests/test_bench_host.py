@@ -1,7 +1,8 @@
 """bench.py's host-side helpers, no GPU: the DRAM-traffic figure is reported
 only for the workload and kernel sources it was captured on, the stress
 sweep's trend test, the workload description, the generator's configuration
-override and the clock sampler (against a stand-in nvidia-smi)."""
+override, the clock sampler (against a stand-in nvidia-smi), and the CPU
+oracle legs: the reference arm's JSON line and the sampled extrapolation."""
 import hashlib
 import os
 
@@ -81,3 +82,46 @@ def test_clock_sampler_without_nvidia_smi(tmp_path, monkeypatch):
     with bench.Clocks(0) as clk:
         pass
     assert clk.summary()["reasons"] == ["unavailable"]
+
+
+def test_reference_arm_runs_on_the_host():
+    # `bench.py --impl reference` times the oracle on the host cores only:
+    # one JSON line with the reference fields, no GPU needed (tiny workload).
+    import json
+    import subprocess
+    import sys
+    env = dict(os.environ, RANK="0")
+    out = subprocess.run([sys.executable, os.path.join(bench.ROOT, "bench.py"), "--impl", "reference",
+                          "--config", "tiny", "--steps", "1", "--warmup", "1"],
+                         capture_output=True, text=True, timeout=600, env=env, cwd=bench.ROOT)
+    assert out.returncode == 0, out.stderr[-2000:]
+    lines = [ln for ln in out.stdout.splitlines() if ln.startswith("{")]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    assert d["impl"] == "reference" and d["value"] > 0 and d["dtype"] == "f32"
+    assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["e2e"]["d2h_bytes_per_step"] == 0
+    assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["cores"] >= 1
+    assert d["steps_timed"] == 1 and d["sample_ms_per_step_measured"] > 0
+
+
+def test_reference_arm_other_ranks_exit_quietly():
+    import subprocess
+    import sys
+    env = dict(os.environ, RANK="1")
+    out = subprocess.run([sys.executable, os.path.join(bench.ROOT, "bench.py"), "--impl", "reference",
+                          "--config", "tiny", "--steps", "1", "--warmup", "1"],
+                         capture_output=True, text=True, timeout=300, env=env, cwd=bench.ROOT)
+    assert out.returncode == 0 and not out.stdout.strip()
+
+
+def test_oracle_sample_extrapolates_every_stage():
+    cfg = synth.CONFIGS["tiny"]
+    q, k, v, _ = synth.make_head(cfg, 0)
+    iq = synth.forgy_init(cfg, q, 0, 0, cfg.Cq)
+    ik = synth.forgy_init(cfg, k, 0, 1, cfg.Ck)
+    sec, desc, stages, meas = bench.oracle_sample(cfg, cfg.rho, q, k, v, iq, ik, rows=256)
+    assert sec > 0 and meas > 0 and "float32" in desc
+    for key in ("kmeans_q_iter", "kmeans_k_iter", "final_assign", "permute", "block_error", "route", "attn"):
+        assert stages[key] >= 0, key
+    # the layer estimate covers every stage of every head
+    assert sec >= cfg.H * (stages["block_error"] + stages["attn"])
