@@ -48,7 +48,10 @@ def forward_heads_sharded(Q, K, V, Cq: int, Ck: int, iters: int, rho: float, sca
         def compute(q, k, v, cq, ck, it, r, s, iq, ik):
             return sv.forward(q, k, v, cq, ck, it, r, s, iq, ik, stream=stream)[0]
     sl = lambda x: None if x is None else x[b:e]
-    part = compute(Q[b:e], K[b:e], V[b:e], Cq, Ck, iters, rho, scale, sl(init_q), sl(init_k))
+    if e > b:
+        part = compute(Q[b:e], K[b:e], V[b:e], Cq, Ck, iters, rho, scale, sl(init_q), sl(init_k))
+    else:  # more ranks than heads: this rank owns none, but joins the gather
+        part = Q.new_empty((0,) + tuple(Q.shape[1:]))
     if not gather or world == 1:
         return part, (b, e)
     # equal-sized blocks for the collective: every rank contributes the

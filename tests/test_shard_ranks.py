@@ -22,9 +22,9 @@ def _free_port():
     return port
 
 
-def _inputs():
+def _inputs(heads=H):
     rng = np.random.default_rng(17)
-    q, k, v = (rng.standard_normal((H, N, D)) for _ in range(3))
+    q, k, v = (rng.standard_normal((heads, N, D)) for _ in range(3))
     return q, k, v, q[:, :CQ].copy(), k[:, :CK].copy()
 
 
@@ -36,7 +36,7 @@ def _oracle_compute(Q, K, V, Cq, Ck, iters, rho, scale, iq, ik):
     return torch.from_numpy(np.stack(outs)) if outs else torch.empty((0,) + tuple(Q.shape[1:]), dtype=Q.dtype)
 
 
-def _rank(rank, world, port, out):
+def _rank(rank, world, port, out, heads=H):
     import datetime
     import torch
     import torch.distributed as dist
@@ -46,7 +46,7 @@ def _rank(rank, world, port, out):
     os.environ["MASTER_PORT"] = str(port)
     dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=60))
     try:
-        q, k, v, iq, ik = (torch.from_numpy(x) for x in _inputs())
+        q, k, v, iq, ik = (torch.from_numpy(x) for x in _inputs(heads))
         O, hr = forward_heads_sharded(q, k, v, CQ, CK, ITERS, RHO, 1 / np.sqrt(D), iq, ik,
                                       compute=_oracle_compute)
         part, _ = forward_heads_sharded(q, k, v, CQ, CK, ITERS, RHO, 1 / np.sqrt(D), iq, ik,
@@ -89,3 +89,26 @@ def test_two_ranks_gather_the_single_process_output():
     for rank, (b, e), O, part in res:
         np.testing.assert_array_equal(O, want)
         np.testing.assert_array_equal(part, want[b:e])
+
+
+def test_more_ranks_than_heads():
+    # one head over two ranks: rank 1 owns no head, computes nothing and still
+    # takes part in the all-gather
+    import torch
+    sys.path.insert(0, ROOT)
+    ctx = mp.get_context("spawn")
+    q_ = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_rank, args=(r, 2, port, q_, 1)) for r in range(2)]
+    for p in procs:
+        p.start()
+    res = sorted((q_.get(timeout=180) for _ in procs), key=lambda x: x[0])
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    q, k, v, iq, ik = (torch.from_numpy(x) for x in _inputs(1))
+    want = _oracle_compute(q, k, v, CQ, CK, ITERS, RHO, 1 / np.sqrt(D), iq, ik).numpy()
+    assert [r[1] for r in res] == [(0, 1), (1, 1)]
+    for rank, (b, e), O, part in res:
+        np.testing.assert_array_equal(O, want)
+        assert part.shape[0] == e - b
